@@ -1,0 +1,189 @@
+/*
+ * fp4lin.h -- C ABI of the B200 (sm_100a) NVFP4 / MXFP4 W4A4 linear layer and
+ * NVFP4 KV cache.
+ *
+ * The formats (web pages cited by title and section):
+ *   - E2M1 elements, 1 sign / 2 exponent / 1 mantissa bit, about -6..6:
+ *     "FP4 auf Blackwell: Was NVFP4 fuer lokale KI wirklich aendert",
+ *     section "Was NVFP4 von frueheren 4-Bit-Formaten unterscheidet";
+ *     "FP8, NVFP4 czy AWQ?", section "Czym roznia sie FP8, NVFP4, MXFP4 i AWQ?".
+ *   - NVFP4: 16-value blocks, one E4M3 (FP8) scale per block plus one FP32
+ *     scale per tensor (same two sections).
+ *   - MXFP4 (OCP Microscaling): 32-value blocks, power-of-two E8M0 scale
+ *     (same two sections).
+ *   - Blockwise Hadamard rotation of the activations, computed online, with
+ *     the rotation folded into the weights: the MR-GPTQ abstract
+ *     (hyper.ai/de/papers/2509.23202), "Abstract".
+ *   - KV cache written in NVFP4, dequantised to FP8 before attention: the
+ *     NVFP4 KV-cache story (hyper.ai/de/stories/...).
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers on the current CUDA device; the
+ *     caller allocates and owns every buffer.  The library allocates no
+ *     memory and keeps no state beyond cached kernel attributes and one
+ *     device status word per device (see fp4lin_device_status).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on it and returns without
+ *     synchronising; results are ready when the stream is.
+ *   - Arguments are checked on the host before anything is launched; on any
+ *     error nothing is launched and a status below is returned.
+ *   - bf16 means IEEE bfloat16 stored as 16-bit words; codes pack two E2M1
+ *     values per byte, element 2i in the low nibble and 2i+1 in the high
+ *     nibble, K (the row) contiguous.
+ *   - "Tensor-core scale layout": scale bytes of a [rows, sf_cols] matrix
+ *     grouped into atoms of 128 rows x 4 scale columns (512 bytes); atom
+ *     (rt, ct) starts at byte (rt * ceil(sf_cols/4) + ct) * 512, and inside
+ *     an atom the scale of row r, column c sits at byte
+ *     (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.  The buffer holds
+ *     fp4lin_scale_bytes(rows, sf_cols) bytes; padding bytes are written 0.
+ *     This is the layout the sm_100 block-scaled tensor-core MMA reads.
+ */
+#ifndef FP4LIN_H
+#define FP4LIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+enum fp4lin_status {
+    FP4LIN_OK = 0,
+    FP4LIN_ERR_INVALID_ARGUMENT = 1, /* null pointer, size <= 0, bad option value */
+    FP4LIN_ERR_UNSUPPORTED_SHAPE = 2, /* a size the kernels do not support (see each call) */
+    FP4LIN_ERR_MISALIGNED = 3,       /* a pointer or leading dimension breaks the 16-byte rule */
+    FP4LIN_ERR_CUDA = 4,             /* a CUDA runtime call or kernel launch failed */
+    FP4LIN_ERR_TIMEOUT = 5,          /* a device-side wait gave up (reported by fp4lin_device_status) */
+    FP4LIN_ERR_DEVICE = 6,           /* the current device is not compute capability 10.0 (B200) */
+    FP4LIN_ERR_WORKSPACE = 7,        /* workspace null or smaller than required */
+    FP4LIN_ERR_OUT_OF_RANGE = 8      /* a KV position outside [0, Lcap) (reported by fp4lin_device_status) */
+};
+
+/* Library version, MAJOR*10000 + MINOR*100 + PATCH. */
+int fp4lin_version(void);
+
+/* Bytes of a tensor-core-layout scale buffer for `rows` rows and `sf_cols`
+ * scale columns: ceil(rows/128)*128 * ceil(sf_cols/4)*4. */
+int64_t fp4lin_scale_bytes(int64_t rows, int64_t sf_cols);
+
+/* Bytes of workspace nvfp4_quantize needs when compute_global_scale = 1
+ * (a constant 4096: one float per partial-maximum block). */
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t cols);
+
+/* Bytes of workspace that lets nvfp4_gemm / mxfp4_gemm split K over more
+ * CTAs for this shape (0 when the shape needs no split).  A smaller
+ * workspace is accepted: the GEMM then runs without the split. */
+size_t fp4lin_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * NVFP4 quantisation of a bf16 matrix, optionally rotated.
+ *
+ *   x       [rows, cols] bf16, row stride ld_x elements.
+ *   hadamard 0 (none) or 16: rotate every 16-value block along the row by
+ *           the Sylvester Hadamard matrix scaled by 1/4 before quantising.
+ *   compute_global_scale
+ *           1: g is OUTPUT -- g = max|x'| / (6*448) over the (rotated)
+ *              tensor, or 1 when that is not > 0; needs `workspace`.
+ *           0: g is INPUT (device float, must be > 0 and finite).
+ *   g       device pointer to one float (the FP32 tensor scale).
+ *   codes   [rows, cols/2] bytes, E2M1 pairs.
+ *   scales  tensor-core scale layout of the [rows, cols/16] E4M3 block
+ *           scales, fp4lin_scale_bytes(rows, cols/16) bytes.
+ * Per 16-value block: t = (amax/6)/g, sf = E4M3 round-to-nearest-even with
+ * saturation at 448, d = dec(sf)*g, r = d > 0 ? 1/d : 0, codes =
+ * E2M1 round-to-nearest-even of x'*r with saturation at 6 (sign kept).
+ * Shapes: rows >= 1, cols a multiple of 64, ld_x >= cols and a multiple of
+ * 8; x, codes, scales 16-byte aligned.
+ */
+int nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                   int hadamard, int compute_global_scale, float *g,
+                   uint8_t *codes, uint8_t *scales,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * y[M, N] = A[M, K] * W[N, K]^T for NVFP4 operands, FP32 accumulation on the
+ * tensor cores, y = bf16_round(g_a * g_w * acc).
+ *   a_codes [M, K/2], a_scales tensor-core layout of [M, K/16];
+ *   w_codes [N, K/2], w_scales tensor-core layout of [N, K/16];
+ *   g_a, g_w device floats; y bf16 with row stride ldy elements.
+ * Shapes: M, N >= 1; K a multiple of 64; ldy >= N and a multiple of 8;
+ * all pointers 16-byte aligned.  workspace may be NULL (see
+ * fp4lin_gemm_workspace_bytes).
+ */
+int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a,
+               const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w,
+               void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * MXFP4 quantisation: 32-value blocks, E8M0 scale byte = clamp(X + 127, 0,
+ * 254) with X = floor(log2 amax) - 2, codes = E2M1 of x' * 2^-X.
+ *   hadamard 0 or 32 (rotate each 32-value block by H_32 / sqrt(32)).
+ *   codes [rows, cols/2]; scales tensor-core layout of [rows, cols/32].
+ * Shapes as nvfp4_quantize.
+ */
+int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                   int hadamard, uint8_t *codes, uint8_t *scales, void *stream);
+
+/* y = A * W^T for MXFP4 operands (E8M0 scales, no tensor scale); otherwise
+ * as nvfp4_gemm. */
+int mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales,
+               const uint8_t *w_codes, const uint8_t *w_scales,
+               void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Append T new K (or V) rows per (batch, head) to an NVFP4 cache.
+ *   kv_new       bf16 [B, H, T, D] contiguous.
+ *   pos          device int32 [B]: row t of batch b goes to position pos[b] + t.
+ *   g            device float, the static FP32 tensor scale (> 0).
+ *   cache_codes  [B, H, Lcap, D/2] bytes.
+ *   cache_scales [B, H, Lcap, D/16] E4M3 bytes, row-major (not the
+ *                tensor-core layout: attention reads the FP8 copy).
+ * Each row is quantised along D exactly like nvfp4_quantize with static g.
+ * A position outside [0, Lcap) is skipped and recorded as
+ * FP4LIN_ERR_OUT_OF_RANGE in the device status word.
+ * Shapes: D a multiple of 16; pointers 16-byte aligned except pos (4).
+ */
+int kv_nvfp4_store(const void *kv_new, const int32_t *pos, const float *g,
+                   uint8_t *cache_codes, uint8_t *cache_scales,
+                   int B, int H, int T, int64_t Lcap, int D, void *stream);
+
+/*
+ * Dequantise the first L positions of every (batch, head) of an NVFP4 cache
+ * to FP8 E4M3 for attention:
+ *   out_fp8[b,h,l,d] = E4M3_rne(e2m1(code) * dec(sf) / 8), out_scale = 8 * g,
+ * so that value = fp8 * out_scale.  The product is exact, so the E4M3
+ * rounding is the only rounding.
+ *   out_fp8 [B, H, L, D] bytes; out_scale device float.
+ * Shapes: 1 <= L <= Lcap; D a multiple of 16; pointers 16-byte aligned
+ * except g and out_scale (4).
+ */
+int kv_nvfp4_load_fp8(const uint8_t *cache_codes, const uint8_t *cache_scales,
+                      const float *g, int64_t L, uint8_t *out_fp8, float *out_scale,
+                      int B, int H, int64_t Lcap, int D, void *stream);
+
+/*
+ * Synchronise `stream`, then read and clear this device's status word.
+ * Returns FP4LIN_OK, or the first device-side error recorded since the last
+ * call (FP4LIN_ERR_TIMEOUT, FP4LIN_ERR_OUT_OF_RANGE), or FP4LIN_ERR_CUDA if
+ * the synchronisation itself failed.
+ */
+int fp4lin_device_status(void *stream);
+
+/*
+ * Diagnostic: run the library's own element conversions on n floats.
+ *   e2m1[i] = E2M1 code (low nibble) of in[i], round-to-nearest-even,
+ *             saturating at 6, sign kept;
+ *   e4m3[i] = E4M3 byte of in[i], round-to-nearest-even, saturating at 448.
+ * These are the device functions every quantiser uses.  n >= 1.
+ */
+int fp4lin_convert_selftest(const float *in, uint8_t *e2m1, uint8_t *e4m3, int64_t n,
+                            void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP4LIN_H */

@@ -1,0 +1,250 @@
+"""Python binding of libfp4lin.so, the B200 (sm_100a) NVFP4 / MXFP4 W4A4 linear
+layer and NVFP4 KV cache.
+
+Argument marshalling only: every step runs in the library's CUDA kernels.
+PyTorch supplies device memory and the current stream.  There is no CPU or
+PyTorch fallback -- if the library cannot be built or loaded, the first call
+raises.
+
+Entry points (same names as the C ABI in include/fp4lin.h):
+  nvfp4_quantize, nvfp4_gemm, mxfp4_quantize, mxfp4_gemm,
+  kv_nvfp4_store, kv_nvfp4_load_fp8
+plus helpers: scale_bytes, gemm_workspace_bytes, device_status,
+convert_selftest, prepare_weight, nvfp4_linear, mxfp4_linear.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+from . import build as _build
+
+__all__ = [
+    "Fp4LinError", "lib", "nvfp4_quantize", "nvfp4_gemm", "mxfp4_quantize", "mxfp4_gemm",
+    "kv_nvfp4_store", "kv_nvfp4_load_fp8", "scale_bytes", "gemm_workspace_bytes",
+    "device_status", "convert_selftest", "QuantizedWeight", "prepare_weight", "nvfp4_linear",
+    "mxfp4_linear", "EXPORTS",
+]
+
+STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA",
+          5: "TIMEOUT", 6: "DEVICE", 7: "WORKSPACE", 8: "OUT_OF_RANGE"}
+
+_i64, _sz, _vp, _int = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int
+EXPORTS = {
+    "fp4lin_version": (_int, []),
+    "fp4lin_scale_bytes": (_i64, [_i64, _i64]),
+    "nvfp4_quantize_workspace_bytes": (_sz, [_i64, _i64]),
+    "fp4lin_gemm_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "nvfp4_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp]),
+    "mxfp4_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp]),
+    "mxfp4_gemm": (_int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp]),
+    "kv_nvfp4_store": (_int, [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _i64, _int, _vp]),
+    "kv_nvfp4_load_fp8": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _int, _int, _i64, _int, _vp]),
+    "fp4lin_device_status": (_int, [_vp]),
+    "fp4lin_convert_selftest": (_int, [_vp, _vp, _vp, _i64, _vp]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Fp4LinError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: FP4LIN_ERR_{STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load (building first if needed) the CUDA library; raises if that is impossible."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            L = ctypes.CDLL(path)
+            for name, (res, args) in EXPORTS.items():
+                fn = getattr(L, name)
+                fn.restype, fn.argtypes = res, args
+            _lib = L
+    return _lib
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(name: str, st: int) -> None:
+    if st != 0:
+        raise Fp4LinError(name, st)
+
+
+def scale_bytes(rows: int, sf_cols: int) -> int:
+    return int(lib().fp4lin_scale_bytes(rows, sf_cols))
+
+
+def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().fp4lin_gemm_workspace_bytes(M, N, K))
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream, return and clear the device status word (0 = OK)."""
+    return int(lib().fp4lin_device_status(_stream(stream)))
+
+
+# ------------------------------------------------------------------ quantisers
+def nvfp4_quantize(x: torch.Tensor, hadamard: int = 0, g: torch.Tensor | None = None, *,
+                   codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                   workspace: torch.Tensor | None = None, stream=None):
+    """NVFP4-quantise bf16 x [rows, cols] (row stride x.stride(0)).
+
+    g None: the FP32 tensor scale is computed (returned as a 1-element device tensor);
+    otherwise g (1-element float32 device tensor) is used as given.
+    Returns (codes uint8 [rows, cols/2], scales uint8 [scale_bytes], g).
+    """
+    rows, cols = x.shape
+    dev = x.device
+    dynamic = g is None
+    if dynamic:
+        g = torch.empty(1, dtype=torch.float32, device=dev)
+        if workspace is None:
+            workspace = torch.empty(int(lib().nvfp4_quantize_workspace_bytes(rows, cols)) // 4,
+                                    dtype=torch.float32, device=dev)
+    if codes is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(scale_bytes(rows, cols // 16), dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("nvfp4_quantize", lib().nvfp4_quantize(
+        _ptr(x), rows, cols, x.stride(0), hadamard, 1 if dynamic else 0, _ptr(g), _ptr(codes), _ptr(scales),
+        _ptr(workspace), ws_bytes, _stream(stream)))
+    return codes, scales, g
+
+
+def mxfp4_quantize(x: torch.Tensor, hadamard: int = 0, *, codes: torch.Tensor | None = None,
+                   scales: torch.Tensor | None = None, stream=None):
+    """MXFP4-quantise bf16 x [rows, cols] -> (codes uint8 [rows, cols/2], scales uint8 [scale_bytes])."""
+    rows, cols = x.shape
+    if codes is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(scale_bytes(rows, cols // 32), dtype=torch.uint8, device=x.device)
+    _check("mxfp4_quantize", lib().mxfp4_quantize(_ptr(x), rows, cols, x.stride(0), hadamard, _ptr(codes),
+                                                  _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+# ------------------------------------------------------------------ GEMMs
+def _gemm_out(M, N, out, dev):
+    return torch.empty(M, N, dtype=torch.bfloat16, device=dev) if out is None else out
+
+
+def _gemm_ws(M, N, K, workspace, dev):
+    if workspace is False:  # explicitly none: the GEMM then runs without splitting K
+        return None, 0
+    if workspace is None:
+        need = gemm_workspace_bytes(M, N, K)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev) if need else None
+    return workspace, (0 if workspace is None else workspace.numel() * workspace.element_size())
+
+
+def nvfp4_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, *, out=None, workspace=None, stream=None):
+    """y [M, N] bf16 = (A_q W_q^T) * g_a * g_w for NVFP4 operands (codes [rows, K/2])."""
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    y = _gemm_out(M, N, out, a_codes.device)
+    ws, wsb = _gemm_ws(M, N, K, workspace, a_codes.device)
+    _check("nvfp4_gemm", lib().nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(g_a), _ptr(w_codes), _ptr(w_scales),
+                                          _ptr(g_w), _ptr(y), M, N, K, y.stride(0), _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
+def mxfp4_gemm(a_codes, a_scales, w_codes, w_scales, *, out=None, workspace=None, stream=None):
+    """y [M, N] bf16 = A_q W_q^T for MXFP4 operands."""
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    y = _gemm_out(M, N, out, a_codes.device)
+    ws, wsb = _gemm_ws(M, N, K, workspace, a_codes.device)
+    _check("mxfp4_gemm", lib().mxfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(w_codes), _ptr(w_scales), _ptr(y),
+                                          M, N, K, y.stride(0), _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
+# ------------------------------------------------------------------ KV cache
+def kv_nvfp4_store(kv_new, pos, g, cache_codes, cache_scales, *, stream=None) -> None:
+    """Quantise kv_new bf16 [B, H, T, D] into cache_codes [B, H, Lcap, D/2] / cache_scales [B, H, Lcap, D/16]
+    at positions pos[b] + t (pos: int32 device [B]; g: float32 device [1])."""
+    B, H, T, D = kv_new.shape
+    Lcap = cache_codes.shape[2]
+    _check("kv_nvfp4_store", lib().kv_nvfp4_store(_ptr(kv_new), _ptr(pos), _ptr(g), _ptr(cache_codes),
+                                                  _ptr(cache_scales), B, H, T, Lcap, D, _stream(stream)))
+
+
+def kv_nvfp4_load_fp8(cache_codes, cache_scales, g, L: int, *, out=None, out_scale=None, stream=None):
+    """Dequantise positions [0, L) to FP8 E4M3 bytes [B, H, L, D]; returns (out, out_scale = 8 g)."""
+    B, H, Lcap, D2 = cache_codes.shape
+    D = D2 * 2
+    dev = cache_codes.device
+    if out is None:
+        out = torch.empty(B, H, L, D, dtype=torch.uint8, device=dev)
+    if out_scale is None:
+        out_scale = torch.empty(1, dtype=torch.float32, device=dev)
+    _check("kv_nvfp4_load_fp8", lib().kv_nvfp4_load_fp8(_ptr(cache_codes), _ptr(cache_scales), _ptr(g), L,
+                                                        _ptr(out), _ptr(out_scale), B, H, Lcap, D, _stream(stream)))
+    return out, out_scale
+
+
+def convert_selftest(x: torch.Tensor, stream=None):
+    """The library's E2M1 and E4M3 conversions of float32 device tensor x (diagnostic)."""
+    n = x.numel()
+    e2 = torch.empty(n, dtype=torch.uint8, device=x.device)
+    e4 = torch.empty(n, dtype=torch.uint8, device=x.device)
+    _check("fp4lin_convert_selftest", lib().fp4lin_convert_selftest(_ptr(x), _ptr(e2), _ptr(e4), n, _stream(stream)))
+    return e2, e4
+
+
+# ------------------------------------------------------------------ layer helpers
+@dataclass
+class QuantizedWeight:
+    """A pre-quantised weight [N, K]: codes, tensor-core-layout scales and (NVFP4) the FP32 scale."""
+    fmt: str
+    codes: torch.Tensor
+    scales: torch.Tensor
+    g: torch.Tensor | None
+    hadamard: int
+    N: int
+    K: int
+
+
+def prepare_weight(w: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0) -> QuantizedWeight:
+    """Quantise a bf16 weight [N, K] once, offline; with hadamard the rotation is folded into it,
+    so y = (x H)(W H)^T = x W^T needs only the online rotation of the activations."""
+    if fmt == "nvfp4":
+        c, s, g = nvfp4_quantize(w, hadamard)
+        return QuantizedWeight("nvfp4", c, s, g, hadamard, w.shape[0], w.shape[1])
+    c, s = mxfp4_quantize(w, hadamard)
+    return QuantizedWeight("mxfp4", c, s, None, hadamard, w.shape[0], w.shape[1])
+
+
+def nvfp4_linear(x: torch.Tensor, w: QuantizedWeight, *, out=None, stream=None) -> torch.Tensor:
+    """y = x W^T: online (rotated) NVFP4 quantisation of x, then the block-scaled GEMM."""
+    c, s, g = nvfp4_quantize(x, w.hadamard, stream=stream)
+    return nvfp4_gemm(c, s, g, w.codes, w.scales, w.g, out=out, stream=stream)
+
+
+def mxfp4_linear(x: torch.Tensor, w: QuantizedWeight, *, out=None, stream=None) -> torch.Tensor:
+    c, s = mxfp4_quantize(x, w.hadamard, stream=stream)
+    return mxfp4_gemm(c, s, w.codes, w.scales, out=out, stream=stream)

@@ -1,0 +1,107 @@
+// common.cuh -- device helpers shared by the quantiser, KV and GEMM kernels
+// (sm_100a only).  Every floating-point step that decides a code uses the
+// explicitly rounded intrinsics (__fmul_rn, __fdiv_rn, __fadd_rn, __fsub_rn),
+// so no multiply-add contraction can change a result.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/fp4lin.h"
+
+namespace fp4lin {
+
+// One status word per device: the first device-side error since it was last
+// read (FP4LIN_ERR_TIMEOUT, FP4LIN_ERR_OUT_OF_RANGE).  Read and cleared by
+// fp4lin_device_status().
+__device__ unsigned int g_device_status;
+
+__device__ __forceinline__ void report_error(unsigned int code)
+{
+    atomicCAS(&g_device_status, 0u, code);
+}
+
+// ------------------------------------------------------------------ loads
+__device__ __forceinline__ uint4 ld_nc_v4(const void *p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void *p)
+{
+    uint2 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void st_v4(void *p, uint4 v)
+{
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Eight bf16 (one 16-byte load) -> eight floats, exact.
+__device__ __forceinline__ void bf16x8_to_f32(uint4 u, float *v)
+{
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// ------------------------------------------------------------------ conversions
+// E2M1 pair: round to nearest even, saturate at +-6, sign kept; `lo` goes to
+// the low nibble (the even element), `hi` to the high nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// Eight floats -> four code bytes (element 0 in the lowest nibble).
+__device__ __forceinline__ uint32_t pack_e2m1x8(const float *v)
+{
+    return cvt_e2m1x2(v[0], v[1]) | (cvt_e2m1x2(v[2], v[3]) << 8) | (cvt_e2m1x2(v[4], v[5]) << 16) |
+           (cvt_e2m1x2(v[6], v[7]) << 24);
+}
+
+// E4M3 byte of a float: round to nearest even, saturate at +-448.
+__device__ __forceinline__ uint32_t cvt_e4m3(float x)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+    return r & 0xFFu;
+}
+
+// Exact value of an E4M3 byte (finite codes; the scale path never makes NaN).
+__device__ __forceinline__ float e4m3_value(uint32_t b)
+{
+    uint32_t e = (b >> 3) & 15u, m = b & 7u;
+    float mag = e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : __fmul_rn((float)m, 0x1p-9f);
+    return (b & 0x80u) ? -mag : mag;
+}
+
+// ------------------------------------------------------------------ misc
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+}  // namespace fp4lin

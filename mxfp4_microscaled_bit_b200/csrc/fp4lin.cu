@@ -1,0 +1,461 @@
+// fp4lin.cu -- the C ABI (include/fp4lin.h): host-side argument checks and
+// launches of the quantiser, KV and GEMM kernels.  One translation unit, so
+// the per-device status word is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm_sm100.cuh"
+#include "kv.cuh"
+#include "quantize.cuh"
+
+using namespace fp4lin;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool probed = false;
+    int status = FP4LIN_OK;
+    int sms = 0;
+    bool gemm_attr[4] = {false, false, false, false};
+};
+
+std::mutex g_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+// Current device's info; FP4LIN_ERR_DEVICE unless it is compute capability 10.0.
+int current_device(DeviceInfo **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return FP4LIN_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FP4LIN_ERR_CUDA;
+        d.status = (major == 10 && minor == 0) ? FP4LIN_OK : FP4LIN_ERR_DEVICE;
+        d.sms = sms;
+        d.probed = true;
+    }
+    *out = &d;
+    return d.status;
+}
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline int launch_status() { return cudaGetLastError() == cudaSuccess ? FP4LIN_OK : FP4LIN_ERR_CUDA; }
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D map over packed codes [rows, K/2] bytes; box = 128 bytes x box_rows, 128-byte swizzle,
+// out-of-range rows and columns read as zero.
+bool make_code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128u, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ GEMM planning
+struct GemmPlan {
+    int bn;
+    int splits, kps, nk, num_mt, num_nt;
+    int64_t ldw;
+    size_t ws_bytes;
+};
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms)
+{
+    GemmPlan p{};
+    p.bn = (M > 128 && N > 128) ? 256 : 64;
+    p.num_mt = (int)((M + 127) / 128);
+    p.num_nt = (int)((N + p.bn - 1) / p.bn);
+    p.nk = (int)((K + 255) / 256);
+    p.splits = 1;
+    p.kps = p.nk;
+    p.ldw = (N + 3) / 4 * 4;
+    const int64_t tiles = (int64_t)p.num_mt * p.num_nt;
+    if (tiles < sms && p.nk >= 2) {
+        int s = (int)std::min<int64_t>({(int64_t)p.nk, std::max<int64_t>(1, sms / tiles), 16});
+        if (s > 1) {
+            const int kps = (p.nk + s - 1) / s;
+            s = (p.nk + kps - 1) / kps;
+            if (s > 1) {
+                p.splits = s;
+                p.kps = kps;
+            }
+        }
+    }
+    p.ws_bytes = p.splits > 1 ? (size_t)p.splits * (size_t)M * (size_t)p.ldw * sizeof(float) : 0;
+    return p;
+}
+
+template <class C>
+int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const uint8_t *a_codes,
+                    const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes, const uint8_t *w_scales,
+                    const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy, float *ws,
+                    cudaStream_t st)
+{
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (!dev->gemm_attr[attr_slot]) {
+            if (cudaFuncSetAttribute(fp4_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM_BYTES) != cudaSuccess)
+                return FP4LIN_ERR_CUDA;
+            dev->gemm_attr[attr_slot] = true;
+        }
+    }
+    CUtensorMap tmA, tmB;
+    if (!make_code_map(&tmA, a_codes, M, K, 128) || !make_code_map(&tmB, w_codes, N, K, C::BN))
+        return FP4LIN_ERR_CUDA;
+    GemmParams p{};
+    p.sfa = a_scales;
+    p.sfb = w_scales;
+    p.g_a = g_a;
+    p.g_w = g_w;
+    p.y = reinterpret_cast<__nv_bfloat16 *>(y);
+    p.ws = ws;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.ldy = ldy;
+    p.ldw = pl.ldw;
+    p.katoms = C::NV ? K / 64 : (K / 32 + 3) / 4;
+    p.num_mt = pl.num_mt;
+    p.num_nt = pl.num_nt;
+    p.nk = pl.nk;
+    p.kps = pl.kps;
+    p.splits = pl.splits;
+    p.work = (int64_t)pl.num_mt * pl.num_nt * pl.splits;
+    const int grid = (int)std::min<int64_t>(p.work, dev->sms);
+    fp4_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, p);
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    if (pl.splits > 1) {
+        const int64_t items = M * ((N + 3) / 4);
+        const int rgrid = (int)std::min<int64_t>((items + 255) / 256, (int64_t)dev->sms * 8);
+        splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(ws, pl.splits, M, N, pl.ldw, C::NV ? g_a : nullptr,
+                                                    C::NV ? g_w : nullptr, reinterpret_cast<__nv_bfloat16 *>(y),
+                                                    ldy);
+        if (launch_status() != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+    }
+    return FP4LIN_OK;
+}
+
+int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
+               const uint8_t *w_scales, const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+               void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!a_codes || !a_scales || !w_codes || !w_scales || !y || (nv && (!g_a || !g_w)))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (M < 1 || N < 1 || K < 1 || ldy < N)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (K % 64 != 0 || ldy % 8 != 0 || M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(a_codes, 16) || !aligned(w_codes, 16) || !aligned(a_scales, 16) || !aligned(w_scales, 16) ||
+        !aligned(y, 16) || (nv && (!aligned(g_a, 4) || !aligned(g_w, 4))) ||
+        (workspace && !aligned(workspace, 16)))
+        return FP4LIN_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    GemmPlan pl = plan_gemm(M, N, K, dev->sms);
+    if (pl.splits > 1 && (!workspace || workspace_bytes < pl.ws_bytes)) {  // no room: run unsplit
+        pl.splits = 1;
+        pl.kps = pl.nk;
+    }
+    float *ws = reinterpret_cast<float *>(workspace);
+    cudaStream_t s = as_stream(stream);
+    if (nv) {
+        if (pl.bn == 256)
+            return launch_gemm_cfg<GemmCfg<256, true>>(dev, 0, pl, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y,
+                                                       M, N, K, ldy, ws, s);
+        return launch_gemm_cfg<GemmCfg<64, true>>(dev, 1, pl, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M,
+                                                  N, K, ldy, ws, s);
+    }
+    if (pl.bn == 256)
+        return launch_gemm_cfg<GemmCfg<256, false>>(dev, 2, pl, a_codes, a_scales, nullptr, w_codes, w_scales,
+                                                     nullptr, y, M, N, K, ldy, ws, s);
+    return launch_gemm_cfg<GemmCfg<64, false>>(dev, 3, pl, a_codes, a_scales, nullptr, w_codes, w_scales, nullptr, y,
+                                                M, N, K, ldy, ws, s);
+}
+
+// ------------------------------------------------------------------ quantiser helpers
+int check_quant_args(const void *x, int64_t rows, int64_t cols, int64_t ld_x, const uint8_t *codes,
+                     const uint8_t *scales)
+{
+    if (!x || !codes || !scales)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (rows < 1 || cols < 1 || ld_x < cols)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (cols % 64 != 0 || ld_x % 8 != 0)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16))
+        return FP4LIN_ERR_MISALIGNED;
+    return FP4LIN_OK;
+}
+
+QuantShape make_shape(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *codes, uint8_t *scales,
+                      int block)
+{
+    QuantShape q{};
+    q.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    q.rows = rows;
+    q.cols = cols;
+    q.ld = ld_x;
+    q.codes = codes;
+    q.scales = scales;
+    q.chunks_per_row = cols / 8;
+    q.total_chunks = rows * (cols / 8);
+    q.sf_cols = cols / block;
+    q.katoms = (q.sf_cols + 3) / 4;
+    const int64_t rows_pad = (rows + 127) / 128 * 128;
+    q.pad_items = rows_pad * q.katoms * 4 - rows * q.sf_cols;
+    return q;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+int fp4lin_version(void) { return 100; }
+
+int64_t fp4lin_scale_bytes(int64_t rows, int64_t sf_cols)
+{
+    if (rows < 1 || sf_cols < 1)
+        return 0;
+    return (rows + 127) / 128 * 128 * ((sf_cols + 3) / 4 * 4);
+}
+
+size_t nvfp4_quantize_workspace_bytes(int64_t, int64_t) { return AMAX_MAX_BLOCKS * sizeof(float); }
+
+size_t fp4lin_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || N < 1 || K < 64)
+        return 0;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            sms = v;
+    } else {
+        cudaGetLastError();
+    }
+    return plan_gemm(M, N, K, sms).ws_bytes;
+}
+
+int nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard, int compute_global_scale,
+                   float *g, uint8_t *codes, uint8_t *scales, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int st = check_quant_args(x, rows, cols, ld_x, codes, scales);
+    if (st != FP4LIN_OK)
+        return st;
+    if (!g || (hadamard != 0 && hadamard != 16) || (compute_global_scale != 0 && compute_global_scale != 1))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (!aligned(g, 4))
+        return FP4LIN_ERR_MISALIGNED;
+    if (compute_global_scale) {
+        if (!workspace || workspace_bytes < AMAX_MAX_BLOCKS * sizeof(float))
+            return FP4LIN_ERR_WORKSPACE;
+        if (!aligned(workspace, 4))
+            return FP4LIN_ERR_MISALIGNED;
+    }
+    DeviceInfo *dev = nullptr;
+    if ((st = current_device(&dev)) != FP4LIN_OK)
+        return st;
+    QuantShape q = make_shape(x, rows, cols, ld_x, codes, scales, 16);
+    cudaStream_t s = as_stream(stream);
+    const int64_t data_blocks = (q.total_chunks + QTHREADS * QUNROLL - 1) / (QTHREADS * QUNROLL);
+    const int64_t grid = data_blocks + (q.pad_items + QTHREADS - 1) / QTHREADS;
+    float *partials = reinterpret_cast<float *>(workspace);
+    int n_partials = 0;
+    if (compute_global_scale) {
+        n_partials = (int)std::min<int64_t>({(q.total_chunks + QTHREADS - 1) / QTHREADS, (int64_t)AMAX_MAX_BLOCKS,
+                                             (int64_t)dev->sms * 4});
+        if (hadamard)
+            nvfp4_amax_kernel<true><<<n_partials, QTHREADS, 0, s>>>(q, partials);
+        else
+            nvfp4_amax_kernel<false><<<n_partials, QTHREADS, 0, s>>>(q, partials);
+        if (launch_status() != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+    }
+    if (hadamard && compute_global_scale)
+        nvfp4_quant_kernel<true, true><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, n_partials, data_blocks);
+    else if (hadamard)
+        nvfp4_quant_kernel<true, false><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, 0, data_blocks);
+    else if (compute_global_scale)
+        nvfp4_quant_kernel<false, true><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, n_partials, data_blocks);
+    else
+        nvfp4_quant_kernel<false, false><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, 0, data_blocks);
+    return launch_status();
+}
+
+int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard, uint8_t *codes,
+                   uint8_t *scales, void *stream)
+{
+    int st = check_quant_args(x, rows, cols, ld_x, codes, scales);
+    if (st != FP4LIN_OK)
+        return st;
+    if (hadamard != 0 && hadamard != 32)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    DeviceInfo *dev = nullptr;
+    if ((st = current_device(&dev)) != FP4LIN_OK)
+        return st;
+    QuantShape q = make_shape(x, rows, cols, ld_x, codes, scales, 32);
+    const int64_t data_blocks = (q.total_chunks + QTHREADS * QUNROLL - 1) / (QTHREADS * QUNROLL);
+    const int64_t grid = data_blocks + (q.pad_items + QTHREADS - 1) / QTHREADS;
+    cudaStream_t s = as_stream(stream);
+    if (hadamard)
+        mxfp4_quant_kernel<true><<<(unsigned)grid, QTHREADS, 0, s>>>(q, data_blocks);
+    else
+        mxfp4_quant_kernel<false><<<(unsigned)grid, QTHREADS, 0, s>>>(q, data_blocks);
+    return launch_status();
+}
+
+int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
+               const uint8_t *w_scales, const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+               void *workspace, size_t workspace_bytes, void *stream)
+{
+    return gemm_entry(true, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N, K, ldy, workspace,
+                      workspace_bytes, stream);
+}
+
+int mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w_codes, const uint8_t *w_scales,
+               void *y, int64_t M, int64_t N, int64_t K, int64_t ldy, void *workspace, size_t workspace_bytes,
+               void *stream)
+{
+    return gemm_entry(false, a_codes, a_scales, nullptr, w_codes, w_scales, nullptr, y, M, N, K, ldy, workspace,
+                      workspace_bytes, stream);
+}
+
+int kv_nvfp4_store(const void *kv_new, const int32_t *pos, const float *g, uint8_t *cache_codes,
+                   uint8_t *cache_scales, int B, int H, int T, int64_t Lcap, int D, void *stream)
+{
+    if (!kv_new || !pos || !g || !cache_codes || !cache_scales)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (B < 1 || H < 1 || T < 1 || Lcap < 1 || D < 1)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (D % 16 != 0)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(kv_new, 16) || !aligned(cache_codes, 16) || !aligned(cache_scales, 16) || !aligned(pos, 4) ||
+        !aligned(g, 4))
+        return FP4LIN_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    KvStoreShape s{};
+    s.x = reinterpret_cast<const __nv_bfloat16 *>(kv_new);
+    s.pos = pos;
+    s.g = g;
+    s.codes = cache_codes;
+    s.scales = cache_scales;
+    s.B = B;
+    s.H = H;
+    s.T = T;
+    s.D = D;
+    s.Lcap = Lcap;
+    s.total_chunks = (int64_t)B * H * T * (D / 8);
+    const int64_t grid = std::min<int64_t>((s.total_chunks + KV_THREADS - 1) / KV_THREADS, (int64_t)dev->sms * 16);
+    kv_store_kernel<<<(unsigned)grid, KV_THREADS, 0, as_stream(stream)>>>(s);
+    return launch_status();
+}
+
+int kv_nvfp4_load_fp8(const uint8_t *cache_codes, const uint8_t *cache_scales, const float *g, int64_t L,
+                      uint8_t *out_fp8, float *out_scale, int B, int H, int64_t Lcap, int D, void *stream)
+{
+    if (!cache_codes || !cache_scales || !g || !out_fp8 || !out_scale)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (B < 1 || H < 1 || L < 1 || Lcap < L || D < 1)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (D % 16 != 0)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(cache_codes, 16) || !aligned(cache_scales, 16) || !aligned(out_fp8, 16) || !aligned(g, 4) ||
+        !aligned(out_scale, 4))
+        return FP4LIN_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    KvLoadShape s{};
+    s.codes = cache_codes;
+    s.scales = cache_scales;
+    s.g = g;
+    s.out = out_fp8;
+    s.out_scale = out_scale;
+    s.L = L;
+    s.Lcap = Lcap;
+    s.bpr = D / 16;
+    s.total_blocks = (int64_t)B * H * L * s.bpr;
+    const int64_t grid = std::min<int64_t>((s.total_blocks + KV_THREADS - 1) / KV_THREADS, (int64_t)dev->sms * 32);
+    kv_load_fp8_kernel<<<(unsigned)grid, KV_THREADS, 0, as_stream(stream)>>>(s);
+    return launch_status();
+}
+
+int fp4lin_device_status(void *stream)
+{
+    if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess)
+        return FP4LIN_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess ||
+        cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+        return FP4LIN_ERR_CUDA;
+    return (int)v;
+}
+
+int fp4lin_convert_selftest(const float *in, uint8_t *e2m1, uint8_t *e4m3, int64_t n, void *stream)
+{
+    if (!in || !e2m1 || !e4m3 || n < 1)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (!aligned(in, 4))
+        return FP4LIN_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    const int64_t grid = std::min<int64_t>((n + 255) / 256, (int64_t)dev->sms * 32);
+    convert_selftest_kernel<<<(unsigned)grid, 256, 0, as_stream(stream)>>>(in, e2m1, e4m3, n);
+    return launch_status();
+}
+
+}  // extern "C"

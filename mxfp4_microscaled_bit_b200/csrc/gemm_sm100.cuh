@@ -1,0 +1,507 @@
+// gemm_sm100.cuh -- y = A W^T for NVFP4 / MXFP4 operands on the sm_100a
+// block-scaled tensor cores (tcgen05.mma kind::mxf4nvf4 / kind::mxf4).
+//
+// The W4A4 layer runs its matrix products on the low-precision tensor cores
+// (page "FP8, NVFP4 czy AWQ?", section "Dlaczego W8A8 i W4A16 to nie to
+// samo?"); Blackwell's 5th-generation tensor cores apply the two-level NVFP4
+// scaling natively (page "FP4 auf Blackwell", section "Was NVFP4 von
+// frueheren 4-Bit-Formaten unterscheidet").
+//
+// Design (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: code tiles by cp.async.bulk.tensor (128-byte
+//               swizzle), scale atoms by cp.async.bulk, into a STAGES-deep
+//               ring of shared-memory stages guarded by mbarriers.
+//   warp 1      owns TMEM; lane 0 copies each stage's scale atoms into TMEM
+//               (tcgen05.cp 32x128b.warpx4) and issues the block-scaled MMAs
+//               (128 x BN x 64 each) into a TMEM accumulator.
+//   warps 2..9  epilogue: tcgen05.ld the accumulator into registers, release
+//               it at once, then scale by g_a*g_w, round to bf16 and store
+//               (or store fp32 partials when K is split across CTAs).
+// Every mbarrier wait is bounded (WAIT_LIMIT_NS); on expiry the kernel
+// records FP4LIN_ERR_TIMEOUT, raises a CTA abort flag, waits (bounded) for
+// its own copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace fp4lin {
+
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;  // 1 s; a tile takes microseconds
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with parity `parity`.  Returns false if it gave
+// up: after WAIT_LIMIT_NS (records a timeout and raises *abort), or, when
+// honor_abort, as soon as another role has raised *abort.
+__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort, bool honor_abort)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 31u) == 0u) {
+            if (honor_abort && *abort)
+                return false;
+            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                report_error(FP4LIN_ERR_TIMEOUT);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// Lane 0 waits, the warp learns the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int lane)
+{
+    int ok = 0;
+    if (lane == 0)
+        ok = wait_bounded(bar, parity, abort, true) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+                 "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+template <bool NV>
+__device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                       uint32_t acc)
+{
+    if constexpr (NV) {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                         d),
+                     "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+                     : "memory");
+    } else {
+        asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                         d),
+                     "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+                     : "memory");
+    }
+}
+
+// 32 consecutive accumulator columns of this thread's TMEM lane, waited for
+// inside the same asm so no register is read early.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+                   "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+                   "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+                   "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, K-major with the 128-byte swizzle: rows of
+// 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Descriptor of one 512-byte scale atom as the tcgen05.cp source: 32 rows of
+// 16 bytes, no swizzle, 8-row core matrices 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+// ------------------------------------------------------------------ configuration
+template <int BN_, bool NV_>
+struct GemmCfg {
+    static constexpr int BN = BN_;
+    static constexpr bool NV = NV_;                       // NVFP4 (16-blocks, E4M3) or MXFP4 (32-blocks, E8M0)
+    static constexpr int BM = 128;
+    static constexpr int BK = 256;                        // elements per stage (128 code bytes per row)
+    static constexpr int MMA_K = 64;
+    static constexpr int APK = NV ? BK / 64 : BK / 128;   // scale atoms per 128 rows per stage
+    static constexpr int RT = BN <= 128 ? 1 : BN / 128;   // 128-row scale tiles per B stage
+    static constexpr int A_BYTES = BM * 128;
+    static constexpr int B_BYTES = BN * 128;
+    static constexpr int SFA_BYTES = APK * 512;
+    static constexpr int SFB_BYTES = RT * APK * 512;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGES = (220 * 1024) / STAGE_BYTES > 8 ? 8 : (220 * 1024) / STAGE_BYTES;
+    static constexpr int NUM_ACC = BN >= 256 ? 1 : 2;
+    static constexpr int SFA_COLS = APK * 4, SFB_COLS = RT * APK * 4;
+    static constexpr int TMEM_USED = NUM_ACC * BN + SFA_COLS + SFB_COLS;
+    static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
+                                   : TMEM_USED <= 256 ? 256 : 512;
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int THREADS = 64 + EPI_WARPS * 32;
+    static constexpr int COLS_PER_WARP = BN / 2;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+    // instruction descriptor: A/B E2M1 (1), dense, K-major, N>>3, scale type, M>>4
+    static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                      ((NV ? 0u : 1u) << 23) | ((uint32_t)(BM >> 4) << 24);
+    static_assert(TMEM_USED <= 512, "TMEM overflow");
+    static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
+    static_assert(STAGES >= 2, "pipeline too shallow");
+};
+
+struct GemmParams {
+    const uint8_t *sfa, *sfb;   // tensor-core scale layouts of A [M, K/blk] and W [N, K/blk]
+    const float *g_a, *g_w;     // NVFP4 tensor scales (null for MXFP4)
+    __nv_bfloat16 *y;
+    float *ws;                  // split-K partials [splits, M, ldw] (splits > 1)
+    int64_t M, N, K, ldy, ldw;
+    int64_t katoms;             // scale atoms per 128-row tile along K
+    int num_mt, num_nt, nk, kps, splits;
+    int64_t work;               // num_mt * num_nt * splits
+};
+
+// MMAs (64 values of K each) in k-tile kt: 4, or fewer in a last partial tile.
+template <class C>
+__device__ __forceinline__ int stage_mmas(int64_t K, int kt)
+{
+    const int64_t left = (K - (int64_t)kt * C::BK) / C::MMA_K;
+    return left < C::BK / C::MMA_K ? (int)left : C::BK / C::MMA_K;
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *bar_area = smem + C::STAGES * C::STAGE_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(bar_area);
+    uint64_t *empty = full + C::STAGES;
+    uint64_t *acc_full = empty + C::STAGES;
+    uint64_t *acc_empty = acc_full + C::NUM_ACC;
+    uint64_t *done_bar = acc_empty + C::NUM_ACC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < C::NUM_ACC; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], C::EPI_WARPS * 32);
+        }
+        mbar_init(done_bar, 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"((uint32_t)C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int64_t tiles_mn = (int64_t)p.num_mt * p.num_nt;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t armed = 0, armed_phase = 0;  // bit s: stage s armed at least once / parity of its last arm
+        for (int64_t w = blockIdx.x; w < p.work; w += gridDim.x) {
+            const int mt = (int)(w % p.num_mt), nt = (int)((w / p.num_mt) % p.num_nt), sp = (int)(w / tiles_mn);
+            const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+            bool ok = true;
+            for (int kt = kt0; kt < kt1 && ok; ++kt) {
+                ok = warp_wait(&empty[stage], phase ^ 1u, abort, lane);
+                if (!ok)
+                    break;
+                if (lane == 0) {
+                    const int mmas = stage_mmas<C>(p.K, kt);
+                    const int atoms = C::NV ? mmas : (mmas + 1) / 2;
+                    uint8_t *sA = smem + stage * C::STAGE_BYTES;
+                    uint8_t *sB = sA + C::A_BYTES;
+                    uint8_t *sSFA = sB + C::B_BYTES;
+                    uint8_t *sSFB = sSFA + C::SFA_BYTES;
+                    mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + C::RT));
+                    armed |= 1u << stage;
+                    armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
+                    tma_load_2d(sA, &tmA, &full[stage], kt * 128, mt * C::BM);
+                    tma_load_2d(sB, &tmB, &full[stage], kt * 128, nt * C::BN);
+                    const int64_t ka = (int64_t)kt * C::APK;
+                    bulk_load(sSFA, p.sfa + ((int64_t)mt * p.katoms + ka) * 512, atoms * 512, &full[stage]);
+                    const int64_t brt0 = ((int64_t)nt * C::BN) / 128;
+#pragma unroll
+                    for (int rt = 0; rt < C::RT; ++rt)
+                        bulk_load(sSFB + rt * C::APK * 512, p.sfb + ((brt0 + rt) * p.katoms + ka) * 512, atoms * 512,
+                                  &full[stage]);
+                }
+                __syncwarp();
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok)
+                break;
+        }
+        // drain: every copy this CTA started has landed before shared memory is released
+        if (lane == 0)
+            for (int s = 0; s < C::STAGES; ++s)
+                if (armed & (1u << s))
+                    wait_bounded(&full[s], (armed_phase >> s) & 1u, abort, false);
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        const uint32_t tm_sfa = tmem_base + C::NUM_ACC * C::BN;
+        const uint32_t tm_sfb = tm_sfa + C::SFA_COLS;
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        bool ok = true;
+        for (int64_t w = blockIdx.x; w < p.work && ok; w += gridDim.x, ++it) {
+            const int nt = (int)((w / p.num_mt) % p.num_nt), sp = (int)(w / tiles_mn);
+            const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+            const int acc = it % C::NUM_ACC;
+            const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
+            ok = warp_wait(&acc_empty[acc], acc_phase ^ 1u, abort, lane);
+            if (!ok)
+                break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + acc * C::BN;
+            // a 64-row B tile reads the second half of its 128-row scale atom at column +2
+            const uint32_t sfb_off = (C::BN == 64 && (((int64_t)nt * 64) & 127)) ? 2u : 0u;
+            for (int kt = kt0; kt < kt1; ++kt) {
+                ok = warp_wait(&full[stage], phase, abort, lane);
+                if (!ok)
+                    break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const int mmas = stage_mmas<C>(p.K, kt);
+                    const int atoms = C::NV ? mmas : (mmas + 1) / 2;
+                    uint8_t *sA = smem + stage * C::STAGE_BYTES;
+                    uint8_t *sB = sA + C::A_BYTES;
+                    uint8_t *sSFA = sB + C::B_BYTES;
+                    uint8_t *sSFB = sSFA + C::SFA_BYTES;
+                    for (int a = 0; a < atoms; ++a) {
+                        tc_cp_atom(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
+                        for (int rt = 0; rt < C::RT; ++rt)
+                            tc_cp_atom(tm_sfb + a * C::RT * 4 + rt * 4,
+                                       desc_sf_atom(smem_u32(sSFB + (rt * C::APK + a) * 512)));
+                    }
+                    const uint64_t dA = desc_sw128(smem_u32(sA)), dB = desc_sw128(smem_u32(sB));
+                    for (int kb = 0; kb < mmas; ++kb) {
+                        uint32_t sfa, sfb, idesc;
+                        if (C::NV) {
+                            sfa = tm_sfa + kb * 4;
+                            sfb = tm_sfb + kb * C::RT * 4 + sfb_off;
+                            idesc = C::IDESC;
+                        } else {
+                            const uint32_t byte = (uint32_t)(kb & 1) * 2u;  // second MMA of an atom: scale bytes 2..3
+                            sfa = (tm_sfa + (kb >> 1) * 4) | (byte << 30);
+                            sfb = (tm_sfb + (kb >> 1) * C::RT * 4 + sfb_off) | (byte << 30);
+                            idesc = C::IDESC | (byte << 29) | (byte << 4);
+                        }
+                        // advance 64 FP4 values = 32 bytes inside the swizzled rows
+                        tc_mma<C::NV>(d_tmem, dA + (uint64_t)(kb * 2), dB + (uint64_t)(kb * 2), idesc, sfa, sfb,
+                                      (kt > kt0 || kb > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok)
+                break;
+            if (lane == 0)
+                tc_commit(&acc_full[acc]);
+            __syncwarp();
+        }
+        // every MMA this CTA issued has completed before TMEM is freed
+        if (lane == 0) {
+            tc_commit(done_bar);
+            wait_bounded(done_bar, 0, abort, false);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------------------- epilogue
+        const int quad = warp & 3;                       // TMEM lanes this warp may access
+        const int half = (warp - 2) >> 2;                // which half of the tile's columns
+        const float gg = C::NV ? __fmul_rn(*p.g_a, *p.g_w) : 1.0f;
+        int it = 0;
+        for (int64_t w = blockIdx.x; w < p.work; w += gridDim.x, ++it) {
+            const int mt = (int)(w % p.num_mt), nt = (int)((w / p.num_mt) % p.num_nt), sp = (int)(w / tiles_mn);
+            const int acc = it % C::NUM_ACC;
+            const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
+            if (!warp_wait(&acc_full[acc], acc_phase, abort, lane))
+                break;
+            tc_fence_after();
+            float v[C::COLS_PER_WARP];
+            const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * C::BN + half * C::COLS_PER_WARP;
+#pragma unroll
+            for (int c = 0; c < C::COLS_PER_WARP; c += 32)
+                tmem_ld32(taddr + c, v + c);
+            tc_fence_before();
+            mbar_arrive(&acc_empty[acc]);  // accumulator free: the next tile's MMAs may start
+
+            const int64_t m = (int64_t)mt * C::BM + quad * 32 + lane;
+            const int64_t n0 = (int64_t)nt * C::BN + half * C::COLS_PER_WARP;
+            if (m < p.M) {
+                if (p.splits == 1) {
+                    __nv_bfloat16 *yr = p.y + m * p.ldy;
+#pragma unroll
+                    for (int c = 0; c < C::COLS_PER_WARP; c += 8) {
+                        const int64_t n = n0 + c;
+                        if (n + 8 <= p.N) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(v[c + 2 * j], gg),
+                                                                          __fmul_rn(v[c + 2 * j + 1], gg));
+                                w4[j] = *reinterpret_cast<uint32_t *>(&b2);
+                            }
+                            st_v4(yr + n, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+                        } else {
+                            for (int j = 0; j < 8; ++j)
+                                if (n + j < p.N)
+                                    yr[n + j] = __float2bfloat16_rn(__fmul_rn(v[c + j], gg));
+                        }
+                    }
+                } else {
+                    float *wr = p.ws + ((int64_t)sp * p.M + m) * p.ldw;
+#pragma unroll
+                    for (int c = 0; c < C::COLS_PER_WARP; c += 4) {
+                        const int64_t n = n0 + c;
+                        if (n + 4 <= p.N) {
+                            st_v4(wr + n, make_uint4(__float_as_uint(v[c]), __float_as_uint(v[c + 1]),
+                                                     __float_as_uint(v[c + 2]), __float_as_uint(v[c + 3])));
+                        } else {
+                            for (int j = 0; j < 4; ++j)
+                                if (n + j < p.N)
+                                    wr[n + j] = v[c + j];
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"((uint32_t)C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// y = bf16(g_a * g_w * sum_s ws[s]) in split order (deterministic).
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *ws, int splits, int64_t M, int64_t N,
+                                                            int64_t ldw, const float *g_a, const float *g_w,
+                                                            __nv_bfloat16 *y, int64_t ldy)
+{
+    const float gg = (g_a && g_w) ? __fmul_rn(*g_a, *g_w) : 1.0f;
+    const int64_t nq = (N + 3) / 4, total = M * nq;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t m = i / nq, n = (i - m * nq) * 4;
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < splits; ++k) {
+            const float *src = ws + ((int64_t)k * M + m) * ldw + n;
+            if (n + 4 <= N) {
+                const float4 f = *reinterpret_cast<const float4 *>(src);
+                s[0] = __fadd_rn(s[0], f.x);
+                s[1] = __fadd_rn(s[1], f.y);
+                s[2] = __fadd_rn(s[2], f.z);
+                s[3] = __fadd_rn(s[3], f.w);
+            } else {
+                for (int j = 0; j < 4 && n + j < N; ++j)
+                    s[j] = __fadd_rn(s[j], src[j]);
+            }
+        }
+        __nv_bfloat16 *dst = y + m * ldy + n;
+        if (n + 4 <= N) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(__fmul_rn(s[0], gg), __fmul_rn(s[1], gg));
+            __nv_bfloat162 hi = __floats2bfloat162_rn(__fmul_rn(s[2], gg), __fmul_rn(s[3], gg));
+            uint2 u = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+            *reinterpret_cast<uint2 *>(dst) = u;
+        } else {
+            for (int j = 0; j < 4 && n + j < N; ++j)
+                dst[j] = __float2bfloat16_rn(__fmul_rn(s[j], gg));
+        }
+    }
+}
+
+}  // namespace fp4lin

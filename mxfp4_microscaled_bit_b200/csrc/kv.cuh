@@ -1,0 +1,125 @@
+// kv.cuh -- NVFP4 KV cache: quantise appended K/V rows into the cache, and
+// dequantise the cache to FP8 E4M3 for attention (the NVFP4 KV-cache story,
+// hyper.ai/de/stories/...: new K/V vectors are written in NVFP4, the KV
+// tensors are dequantised to FP8 before the attention computation).
+#pragma once
+
+#include "common.cuh"
+
+namespace fp4lin {
+
+constexpr int KV_THREADS = 256;
+
+struct KvStoreShape {
+    const __nv_bfloat16 *x;  // [B, H, T, D]
+    const int32_t *pos;      // [B]
+    const float *g;
+    uint8_t *codes, *scales; // [B, H, Lcap, D/2], [B, H, Lcap, D/16]
+    int B, H, T, D;
+    int64_t Lcap;
+    int64_t total_chunks;    // B*H*T*D/8
+};
+
+// One lane per 8 values, a lane pair per 16-value block (as the NVFP4
+// quantiser, without rotation and with the static tensor scale).
+__global__ void __launch_bounds__(KV_THREADS) kv_store_kernel(KvStoreShape s)
+{
+    const int lane = threadIdx.x & 31;
+    const bool upper = lane & 1;
+    const float g = *s.g;
+    const int64_t cpr = s.D / 8;
+    const int64_t stride = (int64_t)gridDim.x * KV_THREADS;
+    for (int64_t w0 = (int64_t)blockIdx.x * KV_THREADS + (threadIdx.x & ~31); w0 < s.total_chunks; w0 += stride) {
+        const int64_t i = w0 + lane;
+        const bool valid = i < s.total_chunks;
+        int64_t row = 0, c8 = 0;
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (valid) {
+            row = i / cpr;
+            c8 = i - row * cpr;
+            raw = ld_nc_v4(s.x + row * s.D + c8 * 8);
+        }
+        float v[8];
+        bf16x8_to_f32(raw, v);
+        float amax = fmaxf(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            amax = fmaxf(amax, fabsf(v[j]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
+        const uint32_t sf = cvt_e4m3(t);
+        const float d = __fmul_rn(e4m3_value(sf), g);
+        const float rcp = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            v[j] = __fmul_rn(v[j], rcp);
+        const uint32_t packed = pack_e2m1x8(v);
+        if (valid) {
+            const int64_t t_idx = row % s.T, bh = row / s.T, b = bh / s.H;
+            const int64_t p = (int64_t)s.pos[b] + t_idx;
+            if (p < 0 || p >= s.Lcap) {
+                if (c8 == 0)
+                    report_error(FP4LIN_ERR_OUT_OF_RANGE);
+                continue;
+            }
+            const int64_t dst = bh * s.Lcap + p;
+            *reinterpret_cast<uint32_t *>(s.codes + dst * (s.D / 2) + c8 * 4) = packed;
+            if (!upper)
+                s.scales[dst * (s.D / 16) + (c8 >> 1)] = (uint8_t)sf;
+        }
+    }
+}
+
+struct KvLoadShape {
+    const uint8_t *codes, *scales;
+    const float *g;
+    uint8_t *out;
+    float *out_scale;
+    int64_t L, Lcap, bpr;  // bpr: 16-value blocks per row (D/16)
+    int64_t total_blocks;  // B*H*L*bpr
+};
+
+// One thread per 16-value block: 8 code bytes + 1 scale byte in, 16 FP8 bytes
+// out.  e2m1 * (dec(sf) / 8) is formed in f16x2: both factors and the product
+// are exact there (at most 6 significant bits, magnitudes in [2^-13, 336]),
+// so the E4M3 rounding of the f16 product is the single rounding.
+__global__ void __launch_bounds__(KV_THREADS) kv_load_fp8_kernel(KvLoadShape s)
+{
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        *s.out_scale = __fmul_rn(8.0f, *s.g);
+    const int64_t stride = (int64_t)gridDim.x * KV_THREADS;
+    for (int64_t i = (int64_t)blockIdx.x * KV_THREADS + threadIdx.x; i < s.total_blocks; i += stride) {
+        const int64_t row = i / s.bpr, blk = i - row * s.bpr;
+        const int64_t bh = row / s.L, l = row - bh * s.L;
+        const int64_t src = bh * s.Lcap + l;
+        const uint2 c = ld_nc_v2(s.codes + src * (s.bpr * 8) + blk * 8);
+        const uint32_t sf = s.scales[src * s.bpr + blk];
+        const __half2 s2 = __float2half2_rn(__fmul_rn(e4m3_value(sf), 0.125f));
+        const uint32_t s2u = *reinterpret_cast<const uint32_t *>(&s2);
+        uint32_t out[4];
+        const uint32_t cw[2] = {c.x, c.y};
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            uint32_t h[4];
+            asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+                "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+                "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+                "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+                "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+                "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+                : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(cw[w]));
+            uint16_t q[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint32_t p;
+                asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(h[k]), "r"(s2u));
+                asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(q[k]) : "r"(p));
+            }
+            out[2 * w] = (uint32_t)q[0] | ((uint32_t)q[1] << 16);
+            out[2 * w + 1] = (uint32_t)q[2] | ((uint32_t)q[3] << 16);
+        }
+        st_v4(s.out + i * 16, make_uint4(out[0], out[1], out[2], out[3]));
+    }
+}
+
+}  // namespace fp4lin

@@ -1,0 +1,109 @@
+"""The C ABI without a GPU: the library builds and loads, exports every entry point
+include/fp4lin.h declares, and its host-side checks return the documented status
+without launching anything (fake device pointers are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mxfp4_microscaled_bit_b200 as fl
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp4lin.h")
+
+OK, INVALID, SHAPE, MISALIGNED, WORKSPACE = 0, 1, 2, 3, 7
+P = 0x10000  # a 16-byte aligned fake device address; never dereferenced on these paths
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|int64_t|size_t)\s+(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) == 12, names
+    L = fl.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(fl.EXPORTS)
+
+
+def test_library_has_no_driver_dependency():
+    # the runtime is linked statically and the driver is reached through an entry-point query,
+    # so the library loads on a host without libcuda
+    out = os.popen(f"ldd {fl.library_path()}").read()
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def test_sizes():
+    L = fl.lib()
+    assert L.fp4lin_version() == 100
+    assert L.fp4lin_scale_bytes(1, 1) == 512
+    assert L.fp4lin_scale_bytes(128, 4) == 512
+    assert L.fp4lin_scale_bytes(129, 8) == 2048
+    assert L.fp4lin_scale_bytes(8192, 256) == 8192 * 256
+    assert L.nvfp4_quantize_workspace_bytes(8192, 4096) == 4096
+    # prefill shape needs no split; decode shapes split K over the SMs
+    assert L.fp4lin_gemm_workspace_bytes(8192, 14336, 4096) == 0
+    assert L.fp4lin_gemm_workspace_bytes(16, 4096, 4096) > 0
+
+
+def q(x=P, rows=16, cols=128, ld=128, had=0, dyn=0, g=P, codes=P, scales=P, ws=P, wsb=4096):
+    return fl.lib().nvfp4_quantize(x, rows, cols, ld, had, dyn, g, codes, scales, ws, wsb, None)
+
+
+def test_nvfp4_quantize_argument_checks():
+    assert q(x=None) == INVALID
+    assert q(codes=None) == INVALID
+    assert q(g=None) == INVALID
+    assert q(rows=0) == INVALID
+    assert q(ld=64) == INVALID
+    assert q(had=8) == INVALID
+    assert q(dyn=2) == INVALID
+    assert q(cols=96, ld=96) == SHAPE
+    assert q(ld=132) == SHAPE
+    assert q(x=P + 8) == MISALIGNED
+    assert q(scales=P + 4) == MISALIGNED
+    assert q(dyn=1, ws=None) == WORKSPACE
+    assert q(dyn=1, wsb=100) == WORKSPACE
+
+
+def test_mxfp4_quantize_argument_checks():
+    L = fl.lib()
+    assert L.mxfp4_quantize(P, 4, 128, 128, 16, P, P, None) == INVALID
+    assert L.mxfp4_quantize(P, 4, 96, 96, 0, P, P, None) == SHAPE
+    assert L.mxfp4_quantize(P + 2, 4, 128, 128, 0, P, P, None) == MISALIGNED
+
+
+def g(M=16, N=64, K=128, ldy=64, a=P, y=P, ga=P):
+    return fl.lib().nvfp4_gemm(a, P, ga, P, P, P, y, M, N, K, ldy, None, 0, None)
+
+
+def test_gemm_argument_checks():
+    assert g(a=None) == INVALID
+    assert g(ga=None) == INVALID
+    assert g(M=0) == INVALID
+    assert g(ldy=32) == INVALID
+    assert g(K=96) == SHAPE
+    assert g(ldy=68, N=66) == SHAPE
+    assert g(y=P + 2) == MISALIGNED
+    L = fl.lib()
+    assert L.mxfp4_gemm(P, P, P, P, P, 16, 64, 96, 64, None, 0, None) == SHAPE
+
+
+def test_kv_argument_checks():
+    L = fl.lib()
+    assert L.kv_nvfp4_store(P, P, P, P, P, 2, 2, 1, 8, 24, None) == SHAPE
+    assert L.kv_nvfp4_store(P, P, P, P, P, 0, 2, 1, 8, 128, None) == INVALID
+    assert L.kv_nvfp4_store(P, P + 2, P, P, P, 2, 2, 1, 8, 128, None) == MISALIGNED
+    assert L.kv_nvfp4_load_fp8(P, P, P, 9, P, P, 2, 2, 8, 128, None) == INVALID  # L > Lcap
+    assert L.kv_nvfp4_load_fp8(P, P, P, 8, P + 1, P, 2, 2, 8, 128, None) == MISALIGNED
+    assert L.fp4lin_convert_selftest(P, P, P, 0, None) == INVALID
+
+
+@pytest.mark.parametrize("fn", ["nvfp4_quantize", "mxfp4_quantize", "nvfp4_gemm", "mxfp4_gemm",
+                                "kv_nvfp4_store", "kv_nvfp4_load_fp8"])
+def test_binding_names_match_abi(fn):
+    assert callable(getattr(fl, fn))

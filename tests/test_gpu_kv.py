@@ -1,0 +1,102 @@
+"""GPU parity of the NVFP4 KV cache (store of new K/V rows, dequantisation to FP8)
+against the oracle, bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import mxfp4_microscaled_bit_b200 as fl
+import synthetic_inputs as si
+from gpu_util import DEV, assert_bytes_equal, status_ok
+
+pytestmark = pytest.mark.gpu
+
+
+def _g_of(x_cpu):
+    return np.float32(np.abs(x_cpu.float().numpy()).max()) / np.float32(2688.0)
+
+
+def test_kv_small_store_and_load(orc):
+    B, H, Lcap, D = 3, 2, 48, 128
+    rng = np.random.default_rng(4)
+    prefill = si.to_bf16(rng.standard_normal((B, H, 30, D)).astype(np.float32) * 2)
+    step = si.to_bf16(rng.standard_normal((B, H, 1, D)).astype(np.float32) * 5)  # exceeds the static scale
+    g = _g_of(prefill)
+    gt = torch.tensor([g], dtype=torch.float32, device=DEV)
+    codes = torch.zeros(B, H, Lcap, D // 2, dtype=torch.uint8, device=DEV)
+    scales = torch.zeros(B, H, Lcap, D // 16, dtype=torch.uint8, device=DEV)
+    oc = np.zeros((B, H, Lcap, D // 2), np.uint8)
+    osf = np.zeros((B, H, Lcap, D // 16), np.uint8)
+    pos0 = np.zeros(B, np.int32)
+    fl.kv_nvfp4_store(prefill.to(DEV), torch.from_numpy(pos0).to(DEV), gt, codes, scales)
+    orc.kv_store(prefill, pos0, g, oc, osf)
+    pos1 = np.array([30, 35, 47], np.int32)  # sequences at different lengths, one at the last slot
+    fl.kv_nvfp4_store(step.to(DEV), torch.from_numpy(pos1).to(DEV), gt, codes, scales)
+    orc.kv_store(step, pos1, g, oc, osf)
+    status_ok()
+    assert_bytes_equal(codes.cpu().numpy(), oc, "cache codes")
+    assert_bytes_equal(scales.cpu().numpy(), osf, "cache scales")
+    for L in (1, 31, 48):
+        out = torch.full((B, H, L, D), 0x7F, dtype=torch.uint8, device=DEV)
+        o, osc = fl.kv_nvfp4_load_fp8(codes, scales, gt, L, out=out)
+        status_ok()
+        assert_bytes_equal(o.cpu().numpy(), orc.kv_load_fp8(oc, osf, L), f"fp8 L={L}")
+        assert osc.item() == np.float32(8.0) * g
+
+
+def test_kv_out_of_range_position_is_reported():
+    B, H, Lcap, D = 2, 1, 8, 32
+    x = torch.ones(B, H, 1, D, dtype=torch.bfloat16, device=DEV)
+    codes = torch.zeros(B, H, Lcap, D // 2, dtype=torch.uint8, device=DEV)
+    scales = torch.zeros(B, H, Lcap, D // 16, dtype=torch.uint8, device=DEV)
+    pos = torch.tensor([3, 8], dtype=torch.int32, device=DEV)  # 8 == Lcap: outside the cache
+    g = torch.tensor([1.0], dtype=torch.float32, device=DEV)
+    fl.kv_nvfp4_store(x, pos, g, codes, scales)
+    assert fl.device_status() == 8  # FP4LIN_ERR_OUT_OF_RANGE, nothing written for batch 1
+    assert fl.device_status() == 0  # cleared by the read
+    assert codes[0, 0, 3].any() and not codes[1].any()
+
+
+@pytest.mark.slow
+def test_kv_full_cache_sampled(orc):
+    """The full cache workload (64 x 8 x 32768 x 128): prefill 32767 tokens, append one per
+    sequence, dequantise all 32768; sampled (b, h) slices and every appended row are checked
+    against the oracle, and the whole output is checked to hold no NaN byte."""
+    B, H, L, D = si.KVCACHE["B"], si.KVCACHE["H"], si.KVCACHE["L"], si.KVCACHE["D"]
+    which = "k"
+    # generate on the host slice by slice, straight into one pinned buffer
+    host = torch.empty(B, H, L, D, dtype=torch.bfloat16).pin_memory()
+    amax = np.float32(0)
+    for b in range(B):
+        for h in range(H):
+            sl = si.kv_slice(which, b, h)
+            amax = max(amax, np.float32(np.abs(sl).max()))
+            host[b, h] = si.to_bf16(sl)
+    g = np.float32(host.float().abs().max().item()) / np.float32(2688.0)
+    gt = torch.tensor([g], dtype=torch.float32, device=DEV)
+    codes = torch.empty(B, H, L, D // 2, dtype=torch.uint8, device=DEV)
+    scales = torch.empty(B, H, L, D // 16, dtype=torch.uint8, device=DEV)
+    dev_x = host.to(DEV, non_blocking=True)
+    fl.kv_nvfp4_store(dev_x[:, :, :L - 1].contiguous(), torch.zeros(B, dtype=torch.int32, device=DEV), gt,
+                      codes, scales)
+    fl.kv_nvfp4_store(dev_x[:, :, L - 1:].contiguous(), torch.full((B,), L - 1, dtype=torch.int32, device=DEV), gt,
+                      codes, scales)
+    del dev_x
+    out, osc = fl.kv_nvfp4_load_fp8(codes, scales, gt, L)
+    status_ok()
+    assert not bool(((out == 0x7F) | (out == 0xFF)).any())
+    # every appended row
+    new = host[:, :, L - 1:L]
+    oc = np.zeros((B, H, 1, D // 2), np.uint8)
+    osf = np.zeros((B, H, 1, D // 16), np.uint8)
+    orc.kv_store(new, np.zeros(B, np.int32), g, oc, osf)
+    assert_bytes_equal(codes[:, :, L - 1:L].cpu().numpy(), oc, "appended codes")
+    assert_bytes_equal(scales[:, :, L - 1:L].cpu().numpy(), osf, "appended scales")
+    # sampled whole slices, store and load
+    for b, h in [(0, 0), (63, 7), (17, 3), (40, 6)]:
+        oc = np.zeros((1, 1, L, D // 2), np.uint8)
+        osf = np.zeros((1, 1, L, D // 16), np.uint8)
+        orc.kv_store(host[b:b + 1, h:h + 1], np.zeros(1, np.int32), g, oc, osf)
+        assert_bytes_equal(codes[b, h].cpu().numpy(), oc[0, 0], f"codes ({b},{h})")
+        assert_bytes_equal(scales[b, h].cpu().numpy(), osf[0, 0], f"scales ({b},{h})")
+        ref = orc.kv_load_fp8(oc, osf, L)
+        assert_bytes_equal(out[b, h].cpu().numpy(), ref[0, 0], f"fp8 ({b},{h})")
