@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 NVFP4 W4A4 linear layer and NVFP4 KV cache.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  * the prefill linear layer, M=8192 tokens, K=4096, N=14336: online NVFP4
+    quantisation of the bf16 activations with the 16-wide blockwise Hadamard
+    rotation and a dynamic FP32 tensor scale, then the block-scaled tcgen05 GEMM
+    against pre-rotated, pre-quantised NVFP4 weights, bf16 out;
+  * the KV-cache decode step on a 64 x 8 x 32768 x 128 cache: append one new
+    K and one new V row per sequence in NVFP4 and dequantise both whole caches
+    to FP8 E4M3 for attention.
+`value` is the layer's TFLOP/s (2*M*N*K over the layer's device time); the
+per-kernel rooflines, the KV and quantiser bandwidths, the MXFP4 variant and the
+CPU oracle baseline are reported beside it.  Usage:
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 it is launched by torch.distributed.run, one rank per GPU; each rank
+runs the same workload on its own GPU (replicas: the path has no exchange
+step), and times are the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic_inputs as si  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+METRIC = "NVFP4 GEMM TFLOP/s (% dense FP4 peak); quantize/KV GB/s (% of HBM)"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), ws
+
+
+def dist_init(backend: str):
+    rank, local, ws = dist_env()
+    if ws > 1 and not torch.distributed.is_initialized():
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+    return rank, local, ws
+
+
+def max_over_ranks(x: float, device="cpu") -> float:
+    """Maximum of a per-rank number over all ranks (identity when not distributed)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.barrier()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        loaded = [s for s in sm if s > 500] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------ workload
+class Workload:
+    """Device-resident inputs and outputs of one step (nothing is allocated while timing)."""
+
+    def __init__(self, fl, dev, with_kv=True):
+        P = si.PREFILL
+        self.M, self.N, self.K = P["M"], P["N"], P["K"]
+        self.fl, self.dev = fl, dev
+        t0 = time.time()
+        self.A_host = si.prefill_A().pin_memory()
+        W = si.prefill_W()
+        self.A = self.A_host.to(dev)
+        self.w = fl.prepare_weight(W.to(dev), "nvfp4", hadamard=16)  # offline: rotated + quantised once
+        self.w_mx = fl.prepare_weight(W.to(dev), "mxfp4", hadamard=32)
+        del W
+        M, K = self.M, self.K
+        self.a_codes = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        self.a_scales = torch.empty(fl.scale_bytes(M, K // 16), dtype=torch.uint8, device=dev)
+        self.a_scales_mx = torch.empty(fl.scale_bytes(M, K // 32), dtype=torch.uint8, device=dev)
+        self.g_a = torch.empty(1, dtype=torch.float32, device=dev)
+        self.q_ws = torch.empty(1024, dtype=torch.float32, device=dev)
+        self.y = torch.empty(M, self.N, dtype=torch.bfloat16, device=dev)
+        self.y_host = torch.empty(M, self.N, dtype=torch.bfloat16).pin_memory()
+        self.setup_s = {"layer": time.time() - t0}
+        self.with_kv = with_kv
+        if with_kv:
+            self._setup_kv()
+
+    def _setup_kv(self):
+        fl, dev = self.fl, self.dev
+        C = si.KVCACHE
+        B, H, L, D = C["B"], C["H"], C["L"], C["D"]
+        self.B, self.H, self.L, self.D = B, H, L, D
+        t0 = time.time()
+        self.cache = {}
+        self.kv_new_host = {}
+        self.kv_new = {}
+        self.kv_g = {}
+        for which in ("k", "v"):
+            host = torch.empty(B, H, L, D, dtype=torch.bfloat16).pin_memory()
+
+            def fill(bh):
+                b, h = divmod(bh, H)
+                host[b, h] = si.to_bf16(si.kv_slice(which, b, h))
+                return float(host[b, h].abs().max().float())
+
+            from concurrent.futures import ThreadPoolExecutor
+            with ThreadPoolExecutor(max(1, min(32, os.cpu_count() or 1))) as ex:
+                amax = max(ex.map(fill, range(B * H)))
+            # static FP32 scale of the whole tensor from its bf16 values (calibration at setup, not timed)
+            g = np.float32(amax) / np.float32(2688.0)
+            codes = torch.empty(B, H, L, D // 2, dtype=torch.uint8, device=dev)
+            scales = torch.empty(B, H, L, D // 16, dtype=torch.uint8, device=dev)
+            gt = torch.tensor([g], dtype=torch.float32, device=dev)
+            x = host.to(dev)
+            # prefill: the first L-1 tokens through the store path
+            fl.kv_nvfp4_store(x[:, :, :L - 1].contiguous(), torch.zeros(B, dtype=torch.int32, device=dev), gt,
+                              codes, scales)
+            self.kv_new_host[which] = host[:, :, L - 1:L].contiguous().pin_memory()
+            self.kv_new[which] = x[:, :, L - 1:L].contiguous()
+            del x, host
+            out = torch.empty(B, H, L, D, dtype=torch.uint8, device=dev)
+            osc = torch.empty(1, dtype=torch.float32, device=dev)
+            self.cache[which] = (codes, scales, out, osc)
+            self.kv_g[which] = gt
+        self.pos = torch.full((B,), L - 1, dtype=torch.int32, device=dev)
+        torch.cuda.synchronize()
+        assert self.fl.device_status() == 0
+        self.setup_s["kv"] = time.time() - t0
+
+    def step(self, ev=None):
+        """One pass of the hot path; `ev` (5 CUDA events) brackets its four parts."""
+        fl = self.fl
+        if ev is not None:
+            ev[0].record()
+        fl.nvfp4_quantize(self.A, 16, self.g_a, compute_global_scale=True, codes=self.a_codes,
+                          scales=self.a_scales, workspace=self.q_ws)
+        if ev is not None:
+            ev[1].record()
+        fl.nvfp4_gemm(self.a_codes, self.a_scales, self.g_a, self.w.codes, self.w.scales, self.w.g, out=self.y,
+                      workspace=False)
+        if ev is not None:
+            ev[2].record()
+        if self.with_kv:
+            for which in ("k", "v"):
+                codes, scales, _, _ = self.cache[which]
+                fl.kv_nvfp4_store(self.kv_new[which], self.pos, self.kv_g[which], codes, scales)
+            if ev is not None:
+                ev[3].record()
+            for which in ("k", "v"):
+                codes, scales, out, osc = self.cache[which]
+                fl.kv_nvfp4_load_fp8(codes, scales, self.kv_g[which], self.L, out=out, out_scale=osc)
+            if ev is not None:
+                ev[4].record()
+
+    LAUNCHES_PER_STEP = 7  # amax + quantise + GEMM + 2 KV stores + 2 KV loads
+
+    def mxfp4_layer(self):
+        fl = self.fl
+        fl.mxfp4_quantize(self.A, 32, codes=self.a_codes, scales=self.a_scales_mx)
+        fl.mxfp4_gemm(self.a_codes, self.a_scales_mx, self.w_mx.codes, self.w_mx.scales, out=self.y,
+                      workspace=False)
+
+    # algorithmic work
+    def flops(self):
+        return 2.0 * self.M * self.N * self.K
+
+    def quant_bytes(self):
+        return self.M * self.K * (2 + 0.5 + 1 / 16)  # one read of A, codes + scales written
+
+    def gemm_min_bytes(self):
+        M, N, K = self.M, self.N, self.K
+        return (M + N) * K * (0.5 + 1 / 16) + 2.0 * M * N
+
+    def kv_load_bytes(self):
+        return 2 * self.B * self.H * self.L * self.D * (0.5 + 1 / 16 + 1.0)  # K and V
+
+    def kv_store_bytes(self):
+        return 2 * self.B * self.H * self.D * (2 + 0.5 + 1 / 16)
+
+
+def time_loop(fn, steps, stream):
+    """CUDA-event time (ms) of `steps` calls of fn on `stream`."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+class OracleLayer:
+    """The oracle as it stands, on this host's cores: the prefill layer on a sample of rows."""
+
+    def __init__(self):
+        import oracle
+        oracle.lib()
+        self.o = oracle
+        W = si.prefill_W()
+        wc, ws, wg = oracle.nvfp4_quantize(W, 16)  # weight preparation is offline, as on the GPU
+        self.Wd = oracle.dequant(wc, ws, "nvfp4", wg)
+
+    def run(self, rows: int):
+        """Quantise rows 0..rows-1 of the activations (H16 rotation, tensor scale of the sample) and
+        multiply them against all weight rows in fp64; returns (TFLOP/s, seconds)."""
+        o = self.o
+        A = si.prefill_A(0, rows)
+        t0 = time.perf_counter()
+        ac, as_, ag = o.nvfp4_quantize(A, 16)
+        y, _ = o.gemm_abt(o.dequant(ac, as_, "nvfp4", ag), self.Wd)
+        dt = time.perf_counter() - t0
+        return 2.0 * rows * si.PREFILL["N"] * si.PREFILL["K"] / dt / 1e12, dt
+
+    def describe(self, rows, dt):
+        return {"cores": self.o.num_threads(), "kind": "oracle",
+                "sample": f"prefill layer, activation rows 0..{rows - 1} of 8192 quantised with the H16 rotation "
+                          f"and multiplied in fp64 against all 14336 pre-quantised weight rows ({dt:.2f} s)"}
+
+
+def cpu_baseline(rows: int = 1024):
+    ol = OracleLayer()
+    v, dt = ol.run(rows)
+    return {"value": v, "unit": "TFLOP/s", **ol.describe(rows, dt)}
+
+
+def reference_arm(args):
+    """The reference arm: the oracle timed on the host cores, one bounded sample per step."""
+    rank, _, ws = dist_env()
+    if rank != 0:
+        return 0
+    ol = OracleLayer()
+    # about 8 ms of fp64 work per row on 8-16 cores: keep the whole run under a couple of minutes
+    rows = int(min(256, max(8, round(45.0 / max(1, args.steps + args.warmup) / 0.008))))
+    for _ in range(args.warmup):
+        ol.run(rows)
+    vals, secs = [], []
+    for _ in range(max(1, args.steps)):
+        v, dt = ol.run(rows)
+        vals.append(v)
+        secs.append(dt)
+    v = statistics.median(vals)
+    d = ol.describe(rows, statistics.median(secs))
+    line = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": config_dict(),
+            "cpu_baseline": {"value": v, "unit": "TFLOP/s", **d},
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict():
+    P, C = si.PREFILL, si.KVCACHE
+    return {"workload": f"prefill NVFP4 W4A4 linear layer M={P['M']} K={P['K']} N={P['N']}, 16-wide Hadamard "
+                        f"rotation, dynamic tensor scale (Student-t nu=3 activations, N(0,0.02^2) weights) + "
+                        f"NVFP4 KV decode step B={C['B']} H={C['H']} L={C['L']} D={C['D']}",
+            "M": P["M"], "N": P["N"], "K": P["K"], "hadamard": 16,
+            "kv": [C["B"], C["H"], C["L"], C["D"]],
+            "l2": "inputs larger than L2: every step streams 6.7 GB of KV cache after the layer, so no layer "
+                  "operand is L2-resident when the next step starts",
+            "parallelism": "replicas"}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-rows", type=int, default=1024)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    rank, local, ws = dist_init("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import mxfp4_microscaled_bit_b200 as fl
+    fl.lib()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    w = Workload(fl, dev)
+    torch.cuda.synchronize()
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        w.step()
+    torch.cuda.synchronize()
+    assert fl.device_status() == 0
+
+    # ---- timed region: exactly `steps` steps, barrier + synchronize on both sides
+    nparts = 5
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nparts)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        w.step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    assert fl.device_status() == 0
+    total_ms = t_start.elapsed_time(t_end)
+    parts = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(nparts - 1)] for e in evs])  # ms
+    q_ms, gemm_ms, st_ms, ld_ms = (float(np.mean(parts[:, j])) for j in range(4))
+    layer_ms = q_ms + gemm_ms
+
+    total_ms_max = max_over_ranks(total_ms, dev)
+    layer_ms_max = max_over_ranks(layer_ms, dev)
+    gemm_ms_max = max_over_ranks(gemm_ms, dev)
+
+    # ---- MXFP4 variant of the same layer (reported, not part of the step)
+    for _ in range(3):
+        w.mxfp4_layer()
+    mx_ms = time_loop(w.mxfp4_layer, 20, stream) / 20
+
+    # ---- end to end through the public API with host buffers: H2D of A and the new K/V rows,
+    #      the step, D2H of y and the FP8 output scales
+    def e2e_step():
+        w.A.copy_(w.A_host, non_blocking=True)
+        for which in ("k", "v"):
+            w.kv_new[which].copy_(w.kv_new_host[which], non_blocking=True)
+        w.step()
+        w.y_host.copy_(w.y, non_blocking=True)
+        osc = [w.cache[k][3] for k in ("k", "v")]
+        return osc
+
+    e2e_osc_host = torch.empty(2, dtype=torch.float32).pin_memory()
+
+    def e2e_full():
+        osc = e2e_step()
+        e2e_osc_host[0:1].copy_(osc[0], non_blocking=True)
+        e2e_osc_host[1:2].copy_(osc[1], non_blocking=True)
+
+    for _ in range(2):
+        e2e_full()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = time_loop(e2e_full, args.e2e_steps, stream) / args.e2e_steps
+    e2e_ms = max_over_ranks(e2e_ms, dev)
+    h2d = w.A.numel() * 2 + sum(w.kv_new[k].numel() * 2 for k in ("k", "v"))
+    d2h = w.y.numel() * 2 + 8
+
+    # ---- results
+    flops = w.flops()
+    sustained_fp4 = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    burst_fp4 = peaks["bf16_tflops"] * FP4_PER_BF16
+    hbm = peaks["hbm_gbs"]
+
+    def hbm_roof(bytes_, ms):
+        gbs = bytes_ / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "traffic": None, "algorithmic_bytes": bytes_, "ms": ms}
+
+    gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
+    rooflines = {
+        "gemm": {"bound": "tensor", "achieved": gemm_tf, "peak": sustained_fp4, "unit": "TFLOP/s",
+                 "frac": gemm_tf / sustained_fp4, "traffic": None, "ms": gemm_ms,
+                 "peak_basis": f"{peak_src} bf16 sustained x {FP4_PER_BF16:g} (dense FP4 : BF16)",
+                 "frac_of_burst_fp4": gemm_tf / burst_fp4, "frac_of_datasheet_9pf": gemm_tf / 9000.0},
+        "kv_load_fp8": hbm_roof(w.kv_load_bytes(), ld_ms),
+        "quantize": hbm_roof(w.quant_bytes(), q_ms),
+        "kv_store": hbm_roof(w.kv_store_bytes(), st_ms),
+    }
+    rooflines["quantize"]["note"] = "2.5625 B/element (one read of A); the dynamic tensor scale reads A twice"
+    rooflines["kv_load_fp8"]["frac_of_8tbs"] = rooflines["kv_load_fp8"]["achieved"] / 8000.0
+    shares = {"quantize": q_ms, "gemm": gemm_ms, "kv_store": st_ms, "kv_load_fp8": ld_ms}
+    dominant = max(shares, key=shares.get)
+    roof = dict(rooflines[dominant])
+    roof["kernel"] = dominant
+
+    layer_tf = ws * flops / (layer_ms_max * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": layer_tf,
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms_max / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": config_dict(),
+        "roofline": roof,
+        "rooflines": rooflines,
+        "step_ms": {"quantize": q_ms, "gemm": gemm_ms, "kv_store": st_ms, "kv_load_fp8": ld_ms,
+                    "layer": layer_ms, "share": {k: v / sum(shares.values()) for k, v in shares.items()}},
+        "metrics": {"layer_tflops": layer_tf, "gemm_tflops": gemm_tf,
+                    "gemm_frac_dense_fp4": gemm_tf / sustained_fp4,
+                    "quantize_gbs": rooflines["quantize"]["achieved"],
+                    "kv_load_gbs": rooflines["kv_load_fp8"]["achieved"],
+                    "kv_store_us": st_ms * 1e3,
+                    "mxfp4_layer_tflops": flops / (mx_ms * 1e-3) / 1e12},
+        "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": Workload.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk,
+        "peaks": {**peaks, "source": peak_src},
+        "setup_s": w.setup_s,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_rows)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    barrier()
+    if torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -107,19 +107,21 @@ def device_status(stream=None) -> int:
 
 # ------------------------------------------------------------------ quantisers
 def nvfp4_quantize(x: torch.Tensor, hadamard: int = 0, g: torch.Tensor | None = None, *,
-                   codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
-                   workspace: torch.Tensor | None = None, stream=None):
+                   compute_global_scale: bool | None = None, codes: torch.Tensor | None = None,
+                   scales: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
     """NVFP4-quantise bf16 x [rows, cols] (row stride x.stride(0)).
 
-    g None: the FP32 tensor scale is computed (returned as a 1-element device tensor);
-    otherwise g (1-element float32 device tensor) is used as given.
+    By default the FP32 tensor scale is computed when g is None (returned as a new 1-element
+    device tensor) and used as given otherwise.  compute_global_scale=True with a g tensor
+    writes the computed scale into that tensor.
     Returns (codes uint8 [rows, cols/2], scales uint8 [scale_bytes], g).
     """
     rows, cols = x.shape
     dev = x.device
-    dynamic = g is None
-    if dynamic:
+    dynamic = (g is None) if compute_global_scale is None else bool(compute_global_scale)
+    if g is None:
         g = torch.empty(1, dtype=torch.float32, device=dev)
+    if dynamic:
         if workspace is None:
             workspace = torch.empty(int(lib().nvfp4_quantize_workspace_bytes(rows, cols)) // 4,
                                     dtype=torch.float32, device=dev)

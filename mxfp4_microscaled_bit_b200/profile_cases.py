@@ -1,0 +1,79 @@
+"""Small, self-contained cases of each kernel for profilers (ncu): each sets up its
+inputs once, then calls one entry point `--iters` times.  Inputs are larger than
+the 126 MB L2 but hold at most a few GB on the device.
+
+  python -m mxfp4_microscaled_bit_b200.profile_cases --case gemm_prefill --iters 3
+cases: gemm_prefill (8192 x 14336 x 4096 NVFP4, 16-wide rotation), gemm_mxfp4,
+gemm_decode (16 x 14336 x 4096), quant_prefill (8192 x 4096 rotated, dynamic
+scale), kv_load (8 x 8 x 32768 x 128 cache to FP8), kv_store.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import sys
+
+import numpy as np
+import torch
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+import mxfp4_microscaled_bit_b200 as fl  # noqa: E402
+import synthetic_inputs as si  # noqa: E402
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", required=True,
+                    choices=["gemm_prefill", "gemm_mxfp4", "gemm_decode", "quant_prefill", "kv_load", "kv_store"])
+    ap.add_argument("--iters", type=int, default=3)
+    a = ap.parse_args()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if a.case in ("gemm_prefill", "gemm_mxfp4", "quant_prefill"):
+        A = si.prefill_A().to(dev)
+        if a.case == "quant_prefill":
+            fn = lambda: fl.nvfp4_quantize(A, 16)  # noqa: E731
+        else:
+            fmt, had = ("nvfp4", 16) if a.case == "gemm_prefill" else ("mxfp4", 32)
+            w = fl.prepare_weight(si.prefill_W().to(dev), fmt, had)
+            if fmt == "nvfp4":
+                ca, sa, ga = fl.nvfp4_quantize(A, 16)
+                y = torch.empty(A.shape[0], w.N, dtype=torch.bfloat16, device=dev)
+                fn = lambda: fl.nvfp4_gemm(ca, sa, ga, w.codes, w.scales, w.g, out=y)  # noqa: E731
+            else:
+                ca, sa = fl.mxfp4_quantize(A, 32)
+                y = torch.empty(A.shape[0], w.N, dtype=torch.bfloat16, device=dev)
+                fn = lambda: fl.mxfp4_gemm(ca, sa, w.codes, w.scales, out=y)  # noqa: E731
+    elif a.case == "gemm_decode":
+        A = si.decode_A(16, 4096).to(dev)
+        w = fl.prepare_weight(si.decode_W(14336, 4096).to(dev), "nvfp4", 0)
+        ca, sa, ga = fl.nvfp4_quantize(A)
+        fn = lambda: fl.nvfp4_gemm(ca, sa, ga, w.codes, w.scales, w.g)  # noqa: E731
+    else:
+        B, H, L, D = 8, 8, si.KVCACHE["L"], si.KVCACHE["D"]
+        x = torch.empty(B, H, L, D, dtype=torch.bfloat16)
+        for b in range(B):
+            for h in range(H):
+                x[b, h] = si.kv_slice_bf16("k", b, h)
+        g = torch.tensor([np.float32(x.abs().max().float().item()) / np.float32(2688.0)], device=dev)
+        codes = torch.empty(B, H, L, D // 2, dtype=torch.uint8, device=dev)
+        scales = torch.empty(B, H, L, D // 16, dtype=torch.uint8, device=dev)
+        xd = x.to(dev)
+        fl.kv_nvfp4_store(xd, torch.zeros(B, dtype=torch.int32, device=dev), g, codes, scales)
+        if a.case == "kv_load":
+            out = torch.empty(B, H, L, D, dtype=torch.uint8, device=dev)
+            fn = lambda: fl.kv_nvfp4_load_fp8(codes, scales, g, L, out=out)  # noqa: E731
+        else:
+            new = xd[:, :, :1].contiguous()
+            pos = torch.full((B,), L - 1, dtype=torch.int32, device=dev)
+            fn = lambda: fl.kv_nvfp4_store(new, pos, g, codes, scales)  # noqa: E731
+    for _ in range(a.iters):
+        fn()
+    torch.cuda.synchronize()
+    assert fl.device_status() == 0
+    print(f"{a.case}: {a.iters} iterations ok")
+
+
+if __name__ == "__main__":
+    main()
