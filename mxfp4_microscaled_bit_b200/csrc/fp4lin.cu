@@ -227,11 +227,35 @@ int check_quant_args(const void *x, int64_t rows, int64_t cols, int64_t ld_x, co
         return FP4LIN_ERR_INVALID_ARGUMENT;
     if (rows < 1 || cols < 1 || ld_x < cols)
         return FP4LIN_ERR_INVALID_ARGUMENT;
-    if (cols % 64 != 0 || ld_x % 8 != 0)
+    if (cols % 64 != 0 || ld_x % 8 != 0 || (rows + QROWS - 1) / QROWS > 65535)
         return FP4LIN_ERR_UNSUPPORTED_SHAPE;
     if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 16))
         return FP4LIN_ERR_MISALIGNED;
     return FP4LIN_OK;
+}
+
+// quantiser grid: x = 256-value row segments, y = groups of QROWS rows
+dim3 quant_grid(const QuantShape &q)
+{
+    return dim3((unsigned)((q.chunks_per_row + 31) / 32), (unsigned)((q.rows + QROWS - 1) / QROWS));
+}
+
+// amax pass: the same mapping, grid-strided down to at most AMAX_MAX_BLOCKS CTAs
+dim3 amax_grid(const QuantShape &q)
+{
+    const dim3 full = quant_grid(q);
+    const unsigned gx = std::min<unsigned>(full.x, AMAX_MAX_BLOCKS);
+    const unsigned gy = std::min<unsigned>(full.y, std::max<unsigned>(1, AMAX_MAX_BLOCKS / gx));
+    return dim3(gx, gy);
+}
+
+int launch_padding(const QuantShape &q, const DeviceInfo *dev, cudaStream_t s)
+{
+    if (q.pad_items == 0)
+        return FP4LIN_OK;
+    const int64_t grid = std::min<int64_t>((q.pad_items + QTHREADS - 1) / QTHREADS, (int64_t)dev->sms * 4);
+    scale_padding_kernel<<<(unsigned)grid, QTHREADS, 0, s>>>(q);
+    return launch_status();
 }
 
 QuantShape make_shape(const void *x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t *codes, uint8_t *scales,
@@ -245,7 +269,6 @@ QuantShape make_shape(const void *x, int64_t rows, int64_t cols, int64_t ld_x, u
     q.codes = codes;
     q.scales = scales;
     q.chunks_per_row = cols / 8;
-    q.total_chunks = rows * (cols / 8);
     q.sf_cols = cols / block;
     q.katoms = (q.sf_cols + 3) / 4;
     const int64_t rows_pad = (rows + 127) / 128 * 128;
@@ -305,29 +328,30 @@ int nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
         return st;
     QuantShape q = make_shape(x, rows, cols, ld_x, codes, scales, 16);
     cudaStream_t s = as_stream(stream);
-    const int64_t data_blocks = (q.total_chunks + QTHREADS * QUNROLL - 1) / (QTHREADS * QUNROLL);
-    const int64_t grid = data_blocks + (q.pad_items + QTHREADS - 1) / QTHREADS;
+    const dim3 grid(quant_grid(q));
     float *partials = reinterpret_cast<float *>(workspace);
     int n_partials = 0;
     if (compute_global_scale) {
-        n_partials = (int)std::min<int64_t>({(q.total_chunks + QTHREADS - 1) / QTHREADS, (int64_t)AMAX_MAX_BLOCKS,
-                                             (int64_t)dev->sms * 4});
+        const dim3 agrid = amax_grid(q);
+        n_partials = (int)(agrid.x * agrid.y);
         if (hadamard)
-            nvfp4_amax_kernel<true><<<n_partials, QTHREADS, 0, s>>>(q, partials);
+            nvfp4_amax_kernel<true><<<agrid, QTHREADS, 0, s>>>(q, partials);
         else
-            nvfp4_amax_kernel<false><<<n_partials, QTHREADS, 0, s>>>(q, partials);
+            nvfp4_amax_kernel<false><<<agrid, QTHREADS, 0, s>>>(q, partials);
         if (launch_status() != FP4LIN_OK)
             return FP4LIN_ERR_CUDA;
     }
     if (hadamard && compute_global_scale)
-        nvfp4_quant_kernel<true, true><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, n_partials, data_blocks);
+        nvfp4_quant_kernel<true, true><<<grid, QTHREADS, 0, s>>>(q, g, partials, n_partials);
     else if (hadamard)
-        nvfp4_quant_kernel<true, false><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, 0, data_blocks);
+        nvfp4_quant_kernel<true, false><<<grid, QTHREADS, 0, s>>>(q, g, partials, 0);
     else if (compute_global_scale)
-        nvfp4_quant_kernel<false, true><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, n_partials, data_blocks);
+        nvfp4_quant_kernel<false, true><<<grid, QTHREADS, 0, s>>>(q, g, partials, n_partials);
     else
-        nvfp4_quant_kernel<false, false><<<(unsigned)grid, QTHREADS, 0, s>>>(q, g, partials, 0, data_blocks);
-    return launch_status();
+        nvfp4_quant_kernel<false, false><<<grid, QTHREADS, 0, s>>>(q, g, partials, 0);
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    return launch_padding(q, dev, s);
 }
 
 int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard, uint8_t *codes,
@@ -342,14 +366,15 @@ int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
     if ((st = current_device(&dev)) != FP4LIN_OK)
         return st;
     QuantShape q = make_shape(x, rows, cols, ld_x, codes, scales, 32);
-    const int64_t data_blocks = (q.total_chunks + QTHREADS * QUNROLL - 1) / (QTHREADS * QUNROLL);
-    const int64_t grid = data_blocks + (q.pad_items + QTHREADS - 1) / QTHREADS;
     cudaStream_t s = as_stream(stream);
+    const dim3 grid(quant_grid(q));
     if (hadamard)
-        mxfp4_quant_kernel<true><<<(unsigned)grid, QTHREADS, 0, s>>>(q, data_blocks);
+        mxfp4_quant_kernel<true><<<grid, QTHREADS, 0, s>>>(q);
     else
-        mxfp4_quant_kernel<false><<<(unsigned)grid, QTHREADS, 0, s>>>(q, data_blocks);
-    return launch_status();
+        mxfp4_quant_kernel<false><<<grid, QTHREADS, 0, s>>>(q);
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    return launch_padding(q, dev, s);
 }
 
 int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
@@ -417,6 +442,8 @@ int kv_nvfp4_load_fp8(const uint8_t *cache_codes, const uint8_t *cache_scales, c
     int st = current_device(&dev);
     if (st != FP4LIN_OK)
         return st;
+    if ((int64_t)B * H > 65535)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
     KvLoadShape s{};
     s.codes = cache_codes;
     s.scales = cache_scales;
@@ -426,9 +453,10 @@ int kv_nvfp4_load_fp8(const uint8_t *cache_codes, const uint8_t *cache_scales, c
     s.L = L;
     s.Lcap = Lcap;
     s.bpr = D / 16;
-    s.total_blocks = (int64_t)B * H * L * s.bpr;
-    const int64_t grid = std::min<int64_t>((s.total_blocks + KV_THREADS - 1) / KV_THREADS, (int64_t)dev->sms * 32);
-    kv_load_fp8_kernel<<<(unsigned)grid, KV_THREADS, 0, as_stream(stream)>>>(s);
+    const int64_t npair = (L * s.bpr + 1) / 2;
+    const int64_t want = std::max<int64_t>(1, (int64_t)dev->sms * 16 / ((int64_t)B * H));
+    const int64_t gx = std::min<int64_t>((npair + KV_THREADS - 1) / KV_THREADS, want);
+    kv_load_fp8_kernel<<<dim3((unsigned)gx, (unsigned)(B * H)), KV_THREADS, 0, as_stream(stream)>>>(s);
     return launch_status();
 }
 

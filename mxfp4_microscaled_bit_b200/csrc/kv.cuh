@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(KV_THREADS) kv_store_kernel(KvStoreShape s)
         }
         float v[8];
         bf16x8_to_f32(raw, v);
-        float amax = fmaxf(0.0f, 0.0f);
+        float amax = 0.0f;
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             amax = fmaxf(amax, fabsf(v[j]));
@@ -76,49 +76,89 @@ struct KvLoadShape {
     uint8_t *out;
     float *out_scale;
     int64_t L, Lcap, bpr;  // bpr: 16-value blocks per row (D/16)
-    int64_t total_blocks;  // B*H*L*bpr
 };
 
-// One thread per 16-value block: 8 code bytes + 1 scale byte in, 16 FP8 bytes
-// out.  e2m1 * (dec(sf) / 8) is formed in f16x2: both factors and the product
-// are exact there (at most 6 significant bits, magnitudes in [2^-13, 336]),
-// so the E4M3 rounding of the f16 product is the single rounding.
+// 16 FP8 bytes of one 16-value block: e2m1 * (dec(sf) / 8) is formed in
+// f16x2, where both factors and the product are exact (at most 6 significant
+// bits, magnitudes in [2^-13, 336]), so the E4M3 rounding of the f16 product
+// is the single rounding.
+__device__ __forceinline__ uint4 kv_block_fp8(uint2 c, uint32_t sf)
+{
+    const __half2 s2 = __float2half2_rn(__fmul_rn(e4m3_value(sf), 0.125f));
+    const uint32_t s2u = *reinterpret_cast<const uint32_t *>(&s2);
+    uint32_t out[4];
+    const uint32_t cw[2] = {c.x, c.y};
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        uint32_t h[4];
+        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+            "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+            "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+            : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(cw[w]));
+        uint16_t q[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint32_t p;
+            asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(h[k]), "r"(s2u));
+            asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(q[k]) : "r"(p));
+        }
+        out[2 * w] = (uint32_t)q[0] | ((uint32_t)q[1] << 16);
+        out[2 * w + 1] = (uint32_t)q[2] | ((uint32_t)q[3] << 16);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// CTA row y = one (batch, head) slice.  The slice's first L cache rows are
+// contiguous, so block j of the slice sits at code byte 8j and scale byte j
+// and its FP8 output at byte 16j: a flat index, no division.  A thread takes
+// a pair of blocks (16 code bytes) per step, two pairs in flight.
 __global__ void __launch_bounds__(KV_THREADS) kv_load_fp8_kernel(KvLoadShape s)
 {
-    if (blockIdx.x == 0 && threadIdx.x == 0)
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         *s.out_scale = __fmul_rn(8.0f, *s.g);
+    const int64_t bh = blockIdx.y;
+    const int64_t nblk = s.L * s.bpr;
+    const uint8_t *codes = s.codes + bh * s.Lcap * s.bpr * 8;
+    const uint8_t *scales = s.scales + bh * s.Lcap * s.bpr;
+    uint8_t *out = s.out + bh * nblk * 16;
+    const bool vec = ((s.Lcap * s.bpr) & 1) == 0;  // slice base 16-byte aligned
+    const int64_t npair = (nblk + 1) / 2;
     const int64_t stride = (int64_t)gridDim.x * KV_THREADS;
-    for (int64_t i = (int64_t)blockIdx.x * KV_THREADS + threadIdx.x; i < s.total_blocks; i += stride) {
-        const int64_t row = i / s.bpr, blk = i - row * s.bpr;
-        const int64_t bh = row / s.L, l = row - bh * s.L;
-        const int64_t src = bh * s.Lcap + l;
-        const uint2 c = ld_nc_v2(s.codes + src * (s.bpr * 8) + blk * 8);
-        const uint32_t sf = s.scales[src * s.bpr + blk];
-        const __half2 s2 = __float2half2_rn(__fmul_rn(e4m3_value(sf), 0.125f));
-        const uint32_t s2u = *reinterpret_cast<const uint32_t *>(&s2);
-        uint32_t out[4];
-        const uint32_t cw[2] = {c.x, c.y};
+    for (int64_t p0 = (int64_t)blockIdx.x * KV_THREADS + threadIdx.x; p0 < npair; p0 += 2 * stride) {
+        uint2 c[4];
+        uint32_t sf[4];
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            uint32_t h[4];
-            asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-                "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-                "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-                "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-                "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-                "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-                : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(cw[w]));
-            uint16_t q[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                uint32_t p;
-                asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(h[k]), "r"(s2u));
-                asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(q[k]) : "r"(p));
+        for (int u = 0; u < 2; ++u) {
+            const int64_t p = p0 + u * stride, j = 2 * p;
+            c[2 * u] = c[2 * u + 1] = make_uint2(0, 0);
+            sf[2 * u] = sf[2 * u + 1] = 0;
+            if (p < npair) {
+                if (vec && j + 1 < nblk) {
+                    const uint4 v = ld_nc_v4(codes + j * 8);
+                    c[2 * u] = make_uint2(v.x, v.y);
+                    c[2 * u + 1] = make_uint2(v.z, v.w);
+                } else {
+                    c[2 * u] = ld_nc_v2(codes + j * 8);
+                    if (j + 1 < nblk)
+                        c[2 * u + 1] = ld_nc_v2(codes + j * 8 + 8);
+                }
+                sf[2 * u] = scales[j];
+                if (j + 1 < nblk)
+                    sf[2 * u + 1] = scales[j + 1];
             }
-            out[2 * w] = (uint32_t)q[0] | ((uint32_t)q[1] << 16);
-            out[2 * w + 1] = (uint32_t)q[2] | ((uint32_t)q[3] << 16);
         }
-        st_v4(s.out + i * 16, make_uint4(out[0], out[1], out[2], out[3]));
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t p = p0 + u * stride, j = 2 * p;
+            if (p < npair) {
+                st_v4(out + j * 16, kv_block_fp8(c[2 * u], sf[2 * u]));
+                if (j + 1 < nblk)
+                    st_v4(out + j * 16 + 16, kv_block_fp8(c[2 * u + 1], sf[2 * u + 1]));
+            }
+        }
     }
 }
 

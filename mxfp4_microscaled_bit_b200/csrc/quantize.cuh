@@ -12,25 +12,29 @@
 // Work mapping: one lane owns 8 consecutive bf16 (one 16-byte load).  A
 // 16-value NVFP4 block is a lane pair, a 32-value MXFP4 block a lane quad;
 // the last Hadamard stages and the block maxima cross lanes with shuffles.
-// A warp reads 512 contiguous bytes per load and writes 128 contiguous code
-// bytes per store.  Requires cols % 64 == 0, so no block or warp-shuffle
-// group straddles a row.
+// A warp reads 512 contiguous bytes of one row per load and writes 128
+// contiguous code bytes per store.  Requires cols % 64 == 0, so no block is
+// cut by the end of a row.
 #pragma once
 
 #include "common.cuh"
 
 namespace fp4lin {
 
-constexpr int QTHREADS = 256;
-constexpr int QUNROLL = 4;        // 16-byte loads in flight per thread
+constexpr int QTHREADS = 256;          // 8 warps
+constexpr int QWARPS = QTHREADS / 32;
+constexpr int QUNROLL = 4;             // rows per warp per pass: four 16-byte loads in flight per lane
+constexpr int QROWS = QWARPS * QUNROLL;  // rows covered by one CTA in one pass (32)
 constexpr int AMAX_MAX_BLOCKS = 1024;
 
+// Mapping: CTA (bx, by) covers the 256-value row segment bx of rows
+// [by*QROWS, by*QROWS + QROWS); warp w handles rows by*QROWS + w + QWARPS*u,
+// lane l the 8 values at column 8*(32*bx + l).  No integer division.
 struct QuantShape {
     const __nv_bfloat16 *x;
     int64_t rows, cols, ld;
     uint8_t *codes, *scales;
     int64_t chunks_per_row;  // cols / 8
-    int64_t total_chunks;    // rows * cols / 8
     int64_t sf_cols;         // cols / block
     int64_t katoms;          // ceil(sf_cols / 4)
     int64_t pad_items;       // padding bytes of the scale layout
@@ -74,12 +78,6 @@ __device__ __forceinline__ float abs_max8(const float *v)
     for (int i = 0; i < 8; ++i)
         m = fmaxf(m, fabsf(v[i]));
     return m;
-}
-
-__device__ __forceinline__ void chunk_rc(const QuantShape &q, int64_t i, int64_t &r, int64_t &c8)
-{
-    r = i / q.chunks_per_row;
-    c8 = i - r * q.chunks_per_row;
 }
 
 // Rotated (when HAD) values of a lane's chunk of a 16-value block.
@@ -131,55 +129,71 @@ __device__ __forceinline__ void zero_scale_padding(const QuantShape &q, int64_t 
 
 // -------------------------------------------------------------------------
 // Pass 1 of the dynamic tensor scale: per-CTA maxima of |x'| into partials[].
+// Grid-strided over segments (x) and row groups (y); at most AMAX_MAX_BLOCKS CTAs.
 template <bool HAD>
 __global__ void __launch_bounds__(QTHREADS) nvfp4_amax_kernel(QuantShape q, float *partials)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const bool upper = lane & 1;
-    const int64_t stride = (int64_t)gridDim.x * QTHREADS;
     float m = 0.0f;
-    // warp-uniform loop: every lane takes part in the shuffles
-    for (int64_t w0 = (int64_t)blockIdx.x * QTHREADS + warp * 32; w0 < q.total_chunks; w0 += stride) {
-        const int64_t i = w0 + lane;
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (i < q.total_chunks) {
-            int64_t r, c8;
-            chunk_rc(q, i, r, c8);
-            raw = ld_nc_v4(q.x + r * q.ld + c8 * 8);
+    for (int64_t seg = blockIdx.x; seg * 32 < q.chunks_per_row; seg += gridDim.x) {
+        const int64_t c8 = seg * 32 + lane;
+        const bool col_ok = c8 < q.chunks_per_row;
+        for (int64_t r0 = (int64_t)blockIdx.y * QROWS; r0 < q.rows; r0 += (int64_t)gridDim.y * QROWS) {
+            uint4 raw[QUNROLL];
+#pragma unroll
+            for (int u = 0; u < QUNROLL; ++u) {
+                const int64_t r = r0 + warp + QWARPS * u;
+                raw[u] = (col_ok && r < q.rows) ? ld_nc_v4(q.x + r * q.ld + c8 * 8) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < QUNROLL; ++u) {
+                float v[8];
+                nvfp4_lane_values<HAD>(raw[u], upper, v);
+                m = fmaxf(m, abs_max8(v));
+            }
         }
-        float v[8];
-        nvfp4_lane_values<HAD>(raw, upper, v);
-        m = fmaxf(m, abs_max8(v));
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1)
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    __shared__ float red[QTHREADS / 32];
+    __shared__ float red[QWARPS];
     if (lane == 0)
         red[warp] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
         float b = 0.0f;
-        for (int k = 0; k < QTHREADS / 32; ++k)
+        for (int k = 0; k < QWARPS; ++k)
             b = fmaxf(b, red[k]);
-        partials[blockIdx.x] = b;
+        partials[blockIdx.y * gridDim.x + blockIdx.x] = b;
     }
 }
 
+// Zero the padding bytes of a tensor-core scale buffer (launched only when there are any).
+__global__ void __launch_bounds__(QTHREADS) scale_padding_kernel(QuantShape q)
+{
+    for (int64_t j = (int64_t)blockIdx.x * QTHREADS + threadIdx.x; j < q.pad_items; j += (int64_t)gridDim.x * QTHREADS)
+        zero_scale_padding(q, j);
+}
+
 // Pass 2: quantise.  DYNAMIC: g = max(partials) / (6*448) (1 if not > 0),
-// written to g_io by CTA 0; otherwise g is read from g_io.
+// written to g_io by CTA (0,0); otherwise g is read from g_io.
 template <bool HAD, bool DYNAMIC>
 __global__ void __launch_bounds__(QTHREADS)
-    nvfp4_quant_kernel(QuantShape q, float *g_io, const float *partials, int n_partials, int64_t data_blocks)
+    nvfp4_quant_kernel(QuantShape q, float *g_io, const float *partials, int n_partials)
 {
     __shared__ float s_g;
-    __shared__ float red[QTHREADS / 32];
+    __shared__ float red[QWARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (blockIdx.x >= data_blocks) {  // trailing CTAs zero the scale padding
-        const int64_t j = (blockIdx.x - data_blocks) * QTHREADS + threadIdx.x;
-        if (j < q.pad_items)
-            zero_scale_padding(q, j);
-        return;
+    const int64_t c8 = (int64_t)blockIdx.x * 32 + lane;
+    const bool col_ok = c8 < q.chunks_per_row;
+    const int64_t r0 = (int64_t)blockIdx.y * QROWS + warp;
+    // issue the loads first; the tensor-scale reduction overlaps them
+    uint4 raw[QUNROLL];
+#pragma unroll
+    for (int u = 0; u < QUNROLL; ++u) {
+        const int64_t r = r0 + QWARPS * u;
+        raw[u] = (col_ok && r < q.rows) ? ld_nc_v4(q.x + r * q.ld + c8 * 8) : make_uint4(0, 0, 0, 0);
     }
     if (DYNAMIC) {
         float m = 0.0f;
@@ -193,13 +207,13 @@ __global__ void __launch_bounds__(QTHREADS)
         __syncthreads();
         if (threadIdx.x == 0) {
             float b = 0.0f;
-            for (int k = 0; k < QTHREADS / 32; ++k)
+            for (int k = 0; k < QWARPS; ++k)
                 b = fmaxf(b, red[k]);
             float g = __fdiv_rn(b, 2688.0f);  // 6 * 448: E2M1 max times E4M3 max
             if (!(g > 0.0f))
                 g = 1.0f;
             s_g = g;
-            if (blockIdx.x == 0)
+            if (blockIdx.x == 0 && blockIdx.y == 0)
                 *g_io = g;
         }
     } else if (threadIdx.x == 0) {
@@ -208,22 +222,9 @@ __global__ void __launch_bounds__(QTHREADS)
     __syncthreads();
     const float g = s_g;
     const bool upper = lane & 1;
-    const int64_t base = (int64_t)blockIdx.x * QTHREADS * QUNROLL + threadIdx.x;
-
-    uint4 raw[QUNROLL];
 #pragma unroll
     for (int u = 0; u < QUNROLL; ++u) {
-        const int64_t i = base + u * QTHREADS;
-        raw[u] = make_uint4(0, 0, 0, 0);
-        if (i < q.total_chunks) {
-            int64_t r, c8;
-            chunk_rc(q, i, r, c8);
-            raw[u] = ld_nc_v4(q.x + r * q.ld + c8 * 8);
-        }
-    }
-#pragma unroll
-    for (int u = 0; u < QUNROLL; ++u) {
-        const int64_t i = base + u * QTHREADS;
+        const int64_t r = r0 + QWARPS * u;
         float v[8];
         nvfp4_lane_values<HAD>(raw[u], upper, v);
         float amax = abs_max8(v);
@@ -236,9 +237,7 @@ __global__ void __launch_bounds__(QTHREADS)
         for (int j = 0; j < 8; ++j)
             v[j] = __fmul_rn(v[j], rcp);
         const uint32_t packed = pack_e2m1x8(v);
-        if (i < q.total_chunks) {
-            int64_t r, c8;
-            chunk_rc(q, i, r, c8);
+        if (col_ok && r < q.rows) {
             *reinterpret_cast<uint32_t *>(q.codes + r * (q.cols / 2) + c8 * 4) = packed;
             if (!upper)
                 q.scales[tc_offset(r, c8 >> 1, q.katoms)] = (uint8_t)sf;
@@ -250,30 +249,21 @@ __global__ void __launch_bounds__(QTHREADS)
 // of the block maximum (= clamp(floor(log2 amax) - 2 + 127, 0, 254) for
 // finite inputs); elements are scaled by 2^(127 - byte), an exact product.
 template <bool HAD>
-__global__ void __launch_bounds__(QTHREADS) mxfp4_quant_kernel(QuantShape q, int64_t data_blocks)
+__global__ void __launch_bounds__(QTHREADS) mxfp4_quant_kernel(QuantShape q)
 {
-    const int lane = threadIdx.x & 31;
-    if (blockIdx.x >= data_blocks) {
-        const int64_t j = (blockIdx.x - data_blocks) * QTHREADS + threadIdx.x;
-        if (j < q.pad_items)
-            zero_scale_padding(q, j);
-        return;
-    }
-    const int64_t base = (int64_t)blockIdx.x * QTHREADS * QUNROLL + threadIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t c8 = (int64_t)blockIdx.x * 32 + lane;
+    const bool col_ok = c8 < q.chunks_per_row;
+    const int64_t r0 = (int64_t)blockIdx.y * QROWS + warp;
     uint4 raw[QUNROLL];
 #pragma unroll
     for (int u = 0; u < QUNROLL; ++u) {
-        const int64_t i = base + u * QTHREADS;
-        raw[u] = make_uint4(0, 0, 0, 0);
-        if (i < q.total_chunks) {
-            int64_t r, c8;
-            chunk_rc(q, i, r, c8);
-            raw[u] = ld_nc_v4(q.x + r * q.ld + c8 * 8);
-        }
+        const int64_t r = r0 + QWARPS * u;
+        raw[u] = (col_ok && r < q.rows) ? ld_nc_v4(q.x + r * q.ld + c8 * 8) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < QUNROLL; ++u) {
-        const int64_t i = base + u * QTHREADS;
+        const int64_t r = r0 + QWARPS * u;
         float v[8];
         mxfp4_lane_values<HAD>(raw[u], lane, v);
         float amax = abs_max8(v);
@@ -286,9 +276,7 @@ __global__ void __launch_bounds__(QTHREADS) mxfp4_quant_kernel(QuantShape q, int
         for (int j = 0; j < 8; ++j)
             v[j] = __fmul_rn(v[j], s);
         const uint32_t packed = pack_e2m1x8(v);
-        if (i < q.total_chunks) {
-            int64_t r, c8;
-            chunk_rc(q, i, r, c8);
+        if (col_ok && r < q.rows) {
             *reinterpret_cast<uint32_t *>(q.codes + r * (q.cols / 2) + c8 * 4) = packed;
             if ((lane & 3) == 0)
                 q.scales[tc_offset(r, c8 >> 2, q.katoms)] = (uint8_t)byte;

@@ -100,3 +100,23 @@ def test_kv_full_cache_sampled(orc):
         assert_bytes_equal(scales[b, h].cpu().numpy(), osf[0, 0], f"scales ({b},{h})")
         ref = orc.kv_load_fp8(oc, osf, L)
         assert_bytes_equal(out[b, h].cpu().numpy(), ref[0, 0], f"fp8 ({b},{h})")
+
+
+@pytest.mark.parametrize("D,Lcap,L", [(16, 37, 37), (48, 21, 20), (128, 9, 5)])
+def test_kv_odd_slice_alignment(orc, D, Lcap, L):
+    # slices whose base is not 16-byte aligned (Lcap * D/16 odd) and odd block counts take the
+    # narrow-load path; both must match the oracle byte for byte
+    B, H = 2, 3
+    rng = np.random.default_rng(D + Lcap)
+    x = si.to_bf16(rng.standard_normal((B, H, Lcap, D)).astype(np.float32))
+    g = _g_of(x)
+    gt = torch.tensor([g], dtype=torch.float32, device=DEV)
+    codes = torch.zeros(B, H, Lcap, D // 2, dtype=torch.uint8, device=DEV)
+    scales = torch.zeros(B, H, Lcap, D // 16, dtype=torch.uint8, device=DEV)
+    fl.kv_nvfp4_store(x.to(DEV), torch.zeros(B, dtype=torch.int32, device=DEV), gt, codes, scales)
+    oc = np.zeros((B, H, Lcap, D // 2), np.uint8)
+    osf = np.zeros((B, H, Lcap, D // 16), np.uint8)
+    orc.kv_store(x, np.zeros(B, np.int32), g, oc, osf)
+    out, _ = fl.kv_nvfp4_load_fp8(codes, scales, gt, L)
+    status_ok()
+    assert_bytes_equal(out.cpu().numpy(), orc.kv_load_fp8(oc, osf, L), "fp8")
