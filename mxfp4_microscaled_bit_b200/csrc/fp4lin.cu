@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -127,6 +128,15 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms)
     return p;
 }
 
+// m-tiles per raster group; FP4LIN_RASTER overrides (tuning experiments).
+int raster_group(int num_mt)
+{
+    const char *e = getenv("FP4LIN_RASTER");
+    const int env = e ? atoi(e) : 0;
+    const int g = env > 0 ? env : 16;
+    return std::max(1, std::min(g, num_mt));
+}
+
 template <class C>
 int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const uint8_t *a_codes,
                     const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes, const uint8_t *w_scales,
@@ -164,6 +174,7 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
     p.kps = pl.kps;
     p.splits = pl.splits;
     p.work = (int64_t)pl.num_mt * pl.num_nt * pl.splits;
+    p.raster = raster_group(pl.num_mt);
     const int grid = (int)std::min<int64_t>(p.work, dev->sms);
     fp4_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, p);
     if (launch_status() != FP4LIN_OK)

@@ -71,7 +71,7 @@ __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volati
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
-        if ((it & 31u) == 0u) {
+        if ((it & 7u) == 0u) {
             if (honor_abort && *abort)
                 return false;
             if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
@@ -83,12 +83,34 @@ __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// One try_wait that may suspend the thread for up to 20 us while the phase is
+// incomplete; it returns as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+                 : "memory");
+    return ok != 0;
+}
+
+// Single-thread wait: the common case inline, the bounded slow path out of line.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    if (mbar_try_wait_hint(bar, parity))
+        return true;
+    return wait_bounded(bar, parity, abort, true);
+}
+
 // Lane 0 waits, the warp learns the outcome.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int lane)
 {
     int ok = 0;
     if (lane == 0)
-        ok = wait_bounded(bar, parity, abort, true) ? 1 : 0;
+        ok = wait_bar(bar, parity, abort) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -195,7 +217,8 @@ struct GemmCfg {
     static constexpr int STAGES = (220 * 1024) / STAGE_BYTES > 8 ? 8 : (220 * 1024) / STAGE_BYTES;
     static constexpr int NUM_ACC = BN >= 256 ? 1 : 2;
     static constexpr int SFA_COLS = APK * 4, SFB_COLS = RT * APK * 4;
-    static constexpr int TMEM_USED = NUM_ACC * BN + SFA_COLS + SFB_COLS;
+    static constexpr int SF_COLS = SFA_COLS + SFB_COLS;          // one stage's scales
+    static constexpr int TMEM_USED = NUM_ACC * BN + 2 * SF_COLS;  // scales double-buffered across k-tiles
     static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                    : TMEM_USED <= 256 ? 256 : 512;
     static constexpr int EPI_WARPS = 8;
@@ -212,6 +235,7 @@ struct GemmCfg {
 };
 
 struct GemmParams {
+    int raster;                 // m-tiles per raster group (num_mt: plain m-fastest order)
     const uint8_t *sfa, *sfb;   // tensor-core scale layouts of A [M, K/blk] and W [N, K/blk]
     const float *g_a, *g_w;     // NVFP4 tensor scales (null for MXFP4)
     __nv_bfloat16 *y;
@@ -228,6 +252,23 @@ __device__ __forceinline__ int stage_mmas(int64_t K, int kt)
 {
     const int64_t left = (K - (int64_t)kt * C::BK) / C::MMA_K;
     return left < C::BK / C::MMA_K ? (int)left : C::BK / C::MMA_K;
+}
+
+// Work item w -> (m tile, n tile, K split).  Tiles are walked in groups of
+// `raster` m-tiles: inside a group m runs fastest, then n, so the CTAs that
+// run at the same time share a few A and B tiles in L2 instead of one B tile
+// being read by every CTA at once.
+__device__ __forceinline__ void tile_coords(const GemmParams &p, int64_t w, int &mt, int &nt, int &sp)
+{
+    const int64_t tiles_mn = (int64_t)p.num_mt * p.num_nt;
+    sp = (int)(w / tiles_mn);
+    const int64_t t = w - (int64_t)sp * tiles_mn;
+    const int64_t group = (int64_t)p.raster * p.num_nt;
+    const int64_t g = t / group, idx = t - g * group;
+    const int64_t m0 = g * p.raster;
+    const int64_t rows = min((int64_t)p.raster, (int64_t)p.num_mt - m0);
+    mt = (int)(m0 + idx % rows);
+    nt = (int)(idx / rows);
 }
 
 template <class C>
@@ -270,22 +311,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int64_t tiles_mn = (int64_t)p.num_mt * p.num_nt;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- producer
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t armed = 0, armed_phase = 0;  // bit s: stage s armed at least once / parity of its last arm
-        for (int64_t w = blockIdx.x; w < p.work; w += gridDim.x) {
-            const int mt = (int)(w % p.num_mt), nt = (int)((w / p.num_mt) % p.num_nt), sp = (int)(w / tiles_mn);
-            const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+        // ---------------------------------------------------------------- producer (one thread)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t armed = 0, armed_phase = 0;  // bit s: stage s armed at least once / parity of its last arm
             bool ok = true;
-            for (int kt = kt0; kt < kt1 && ok; ++kt) {
-                ok = warp_wait(&empty[stage], phase ^ 1u, abort, lane);
-                if (!ok)
-                    break;
-                if (lane == 0) {
+            for (int64_t w = blockIdx.x; w < p.work && ok; w += gridDim.x) {
+                int mt, nt, sp;
+                tile_coords(p, w, mt, nt, sp);
+                const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+                const int64_t brt0 = ((int64_t)nt * C::BN) / 128;
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    if (!(ok = wait_bar(&empty[stage], phase ^ 1u, abort)))
+                        break;
                     const int mmas = stage_mmas<C>(p.K, kt);
                     const int atoms = C::NV ? mmas : (mmas + 1) / 2;
                     uint8_t *sA = smem + stage * C::STAGE_BYTES;
@@ -299,67 +340,65 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     tma_load_2d(sB, &tmB, &full[stage], kt * 128, nt * C::BN);
                     const int64_t ka = (int64_t)kt * C::APK;
                     bulk_load(sSFA, p.sfa + ((int64_t)mt * p.katoms + ka) * 512, atoms * 512, &full[stage]);
-                    const int64_t brt0 = ((int64_t)nt * C::BN) / 128;
 #pragma unroll
                     for (int rt = 0; rt < C::RT; ++rt)
                         bulk_load(sSFB + rt * C::APK * 512, p.sfb + ((brt0 + rt) * p.katoms + ka) * 512, atoms * 512,
                                   &full[stage]);
-                }
-                __syncwarp();
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
-            if (!ok)
-                break;
-        }
-        // drain: every copy this CTA started has landed before shared memory is released
-        if (lane == 0)
+            // drain: every copy this CTA started has landed before shared memory is released
             for (int s = 0; s < C::STAGES; ++s)
                 if (armed & (1u << s))
                     wait_bounded(&full[s], (armed_phase >> s) & 1u, abort, false);
+        }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        const uint32_t tm_sfa = tmem_base + C::NUM_ACC * C::BN;
-        const uint32_t tm_sfb = tm_sfa + C::SFA_COLS;
-        int stage = 0;
-        uint32_t phase = 0;
-        int it = 0;
-        bool ok = true;
-        for (int64_t w = blockIdx.x; w < p.work && ok; w += gridDim.x, ++it) {
-            const int nt = (int)((w / p.num_mt) % p.num_nt), sp = (int)(w / tiles_mn);
-            const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
-            const int acc = it % C::NUM_ACC;
-            const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
-            ok = warp_wait(&acc_empty[acc], acc_phase ^ 1u, abort, lane);
-            if (!ok)
-                break;
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + acc * C::BN;
-            // a 64-row B tile reads the second half of its 128-row scale atom at column +2
-            const uint32_t sfb_off = (C::BN == 64 && (((int64_t)nt * 64) & 127)) ? 2u : 0u;
-            for (int kt = kt0; kt < kt1; ++kt) {
-                ok = warp_wait(&full[stage], phase, abort, lane);
-                if (!ok)
+        // ---------------------------------------------------------------- MMA issuer (one thread)
+        if (lane == 0) {
+            const uint32_t tm_sf = tmem_base + C::NUM_ACC * C::BN;
+            int stage = 0;
+            uint32_t phase = 0, sfsel = 0;  // sfsel alternates the scale region every k-tile
+            int it = 0;
+            bool ok = true;
+            for (int64_t w = blockIdx.x; w < p.work && ok; w += gridDim.x, ++it) {
+                int mt, nt, sp;
+                tile_coords(p, w, mt, nt, sp);
+                const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+                const int acc = it % C::NUM_ACC;
+                const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
+                if (!(ok = wait_bar(&acc_empty[acc], acc_phase ^ 1u, abort)))
                     break;
-                tc_fence_after();
-                if (lane == 0) {
+                tc_fence_after();  // order the epilogue's TMEM reads before these MMAs
+                const uint32_t d_tmem = tmem_base + acc * C::BN;
+                // a 64-row B tile reads the second half of its 128-row scale atom at column +2
+                const uint32_t sfb_off = (C::BN == 64 && (((int64_t)nt * 64) & 127)) ? 2u : 0u;
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    if (!(ok = wait_bar(&full[stage], phase, abort)))
+                        break;
                     const int mmas = stage_mmas<C>(p.K, kt);
-                    const int atoms = C::NV ? mmas : (mmas + 1) / 2;
                     uint8_t *sA = smem + stage * C::STAGE_BYTES;
                     uint8_t *sB = sA + C::A_BYTES;
                     uint8_t *sSFA = sB + C::B_BYTES;
                     uint8_t *sSFB = sSFA + C::SFA_BYTES;
-                    for (int a = 0; a < atoms; ++a) {
-                        tc_cp_atom(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
-                        for (int rt = 0; rt < C::RT; ++rt)
-                            tc_cp_atom(tm_sfb + a * C::RT * 4 + rt * 4,
-                                       desc_sf_atom(smem_u32(sSFB + (rt * C::APK + a) * 512)));
-                    }
+                    const uint32_t tm_sfa = tm_sf + sfsel * C::SF_COLS;
+                    sfsel ^= 1u;
+                    const uint32_t tm_sfb = tm_sfa + C::SFA_COLS;
                     const uint64_t dA = desc_sw128(smem_u32(sA)), dB = desc_sw128(smem_u32(sB));
                     for (int kb = 0; kb < mmas; ++kb) {
+                        // copy an atom's scales just before the first MMA that reads them, so the
+                        // copies of k-block kb+1 overlap the MMA of k-block kb
+                        const int a = C::NV ? kb : kb >> 1;
+                        if (C::NV || (kb & 1) == 0) {
+                            tc_cp_atom(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
+#pragma unroll
+                            for (int rt = 0; rt < C::RT; ++rt)
+                                tc_cp_atom(tm_sfb + a * C::RT * 4 + rt * 4,
+                                           desc_sf_atom(smem_u32(sSFB + (rt * C::APK + a) * 512)));
+                        }
                         uint32_t sfa, sfb, idesc;
                         if (C::NV) {
                             sfa = tm_sfa + kb * 4;
@@ -367,8 +406,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             idesc = C::IDESC;
                         } else {
                             const uint32_t byte = (uint32_t)(kb & 1) * 2u;  // second MMA of an atom: scale bytes 2..3
-                            sfa = (tm_sfa + (kb >> 1) * 4) | (byte << 30);
-                            sfb = (tm_sfb + (kb >> 1) * C::RT * 4 + sfb_off) | (byte << 30);
+                            sfa = (tm_sfa + a * 4) | (byte << 30);
+                            sfb = (tm_sfb + a * C::RT * 4 + sfb_off) | (byte << 30);
                             idesc = C::IDESC | (byte << 29) | (byte << 4);
                         }
                         // advance 64 FP4 values = 32 bytes inside the swizzled rows
@@ -376,21 +415,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                                       (kt > kt0 || kb > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty[stage]);
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
-                __syncwarp();
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (!ok)
-                break;
-            if (lane == 0)
+                if (!ok)
+                    break;
                 tc_commit(&acc_full[acc]);
-            __syncwarp();
-        }
-        // every MMA this CTA issued has completed before TMEM is freed
-        if (lane == 0) {
+            }
+            // every MMA this CTA issued has completed before TMEM is freed
             tc_commit(done_bar);
             wait_bounded(done_bar, 0, abort, false);
         }
@@ -402,7 +436,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const float gg = C::NV ? __fmul_rn(*p.g_a, *p.g_w) : 1.0f;
         int it = 0;
         for (int64_t w = blockIdx.x; w < p.work; w += gridDim.x, ++it) {
-            const int mt = (int)(w % p.num_mt), nt = (int)((w / p.num_mt) % p.num_nt), sp = (int)(w / tiles_mn);
+            int mt, nt, sp;
+            tile_coords(p, w, mt, nt, sp);
             const int acc = it % C::NUM_ACC;
             const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
             if (!warp_wait(&acc_full[acc], acc_phase, abort, lane))
