@@ -183,6 +183,31 @@ int fp4lin_device_status(void *stream);
 int fp4lin_convert_selftest(const float *in, uint8_t *e2m1, uint8_t *e4m3, int64_t n,
                             void *stream);
 
+/*
+ * nvfp4_quantize with the tensor scale computed (compute_global_scale = 1),
+ * for callers that cannot allocate device memory: plug-ins whose host
+ * framework owns the whole device memory pool and forbids raw cudaMalloc, or
+ * latency-critical loops where a cudaMalloc/cudaFree would synchronise the
+ * device.  The paper has no counterpart: this is an interface convenience.
+ *
+ * Instead of a caller workspace, the per-CTA maxima of the tensor-scale pass
+ * live in a fixed array inside the library: 1024 floats (4 KB) that every
+ * device which loads the library holds until the process exits.  The pass uses
+ * at most 1024 CTAs, so every shape nvfp4_quantize accepts fits; a grid that
+ * would need more partials is rejected with FP4LIN_ERR_UNSUPPORTED_SHAPE.
+ * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
+ * routine).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  All calls on a device share the array and it keeps the last
+ * call's contents (nothing in it has to start at zero: each call overwrites
+ * every partial it reads), so calls that overlap on the GPU -- on different
+ * streams without ordering -- race and must be avoided.
+ * Arguments, results and errors otherwise as nvfp4_quantize; g is OUTPUT.
+ */
+int nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                           int hadamard, float *g, uint8_t *codes, uint8_t *scales,
+                           void *stream);
+
 #ifdef __cplusplus
 }
 #endif

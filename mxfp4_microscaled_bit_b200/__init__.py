@@ -47,6 +47,7 @@ EXPORTS = {
     "kv_nvfp4_load_fp8": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _int, _int, _i64, _int, _vp]),
     "fp4lin_device_status": (_int, [_vp]),
     "fp4lin_convert_selftest": (_int, [_vp, _vp, _vp, _i64, _vp]),
+    "nvfp4_quantize_noalloc": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
 }
 
 _lock = threading.Lock()
@@ -134,6 +135,16 @@ def nvfp4_quantize(x: torch.Tensor, hadamard: int = 0, g: torch.Tensor | None = 
         _ptr(x), rows, cols, x.stride(0), hadamard, 1 if dynamic else 0, _ptr(g), _ptr(codes), _ptr(scales),
         _ptr(workspace), ws_bytes, _stream(stream)))
     return codes, scales, g
+
+
+def nvfp4_quantize_noalloc(x: torch.Tensor, hadamard: int, g: torch.Tensor, codes: torch.Tensor,
+                           scales: torch.Tensor, stream=None) -> None:
+    """nvfp4_quantize with the computed tensor scale, without any device allocation: the library's
+    own 4 KB array holds the tensor-scale partials (see include/fp4lin.h).  The caller passes every
+    output buffer; concurrent calls on one device must not overlap on the GPU."""
+    rows, cols = x.shape
+    _check("nvfp4_quantize_noalloc", lib().nvfp4_quantize_noalloc(
+        _ptr(x), rows, cols, x.stride(0), hadamard, _ptr(g), _ptr(codes), _ptr(scales), _stream(stream)))
 
 
 def mxfp4_quantize(x: torch.Tensor, hadamard: int = 0, *, codes: torch.Tensor | None = None,

@@ -497,4 +497,85 @@ int fp4lin_convert_selftest(const float *in, uint8_t *e2m1, uint8_t *e4m3, int64
     return launch_status();
 }
 
+// ==================================================================== allocation-free variant
+//
+// nvfp4_quantize_noalloc: for callers that cannot allocate device memory --
+// plug-ins whose host framework owns the whole device memory pool and forbids
+// raw cudaMalloc, or latency-critical loops where a cudaMalloc/cudaFree would
+// synchronise the device.  The per-CTA maxima of the tensor-scale pass live in
+// this file-scope array instead of a caller workspace: 1024 floats (4 KB),
+// held by every device that loads the library until the process exits.
+
+}  // extern "C"
+
+static __device__ __align__(256) float g_noalloc_partials[AMAX_MAX_BLOCKS];
+
+namespace {
+
+std::mutex g_noalloc_mutex;
+float *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_partials on device `dev` (the current device).  In
+// host code the symbol is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress, once per device, and cached.
+int noalloc_scratch(int dev, float **out)
+{
+    std::lock_guard<std::mutex> lk(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || p == nullptr)
+            return FP4LIN_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return FP4LIN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard, float *g,
+                           uint8_t *codes, uint8_t *scales, void *stream)
+{
+    int st = check_quant_args(x, rows, cols, ld_x, codes, scales);
+    if (st != FP4LIN_OK)
+        return st;
+    if (!g || (hadamard != 0 && hadamard != 16))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (!aligned(g, 4))
+        return FP4LIN_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    if ((st = current_device(&dev)) != FP4LIN_OK)
+        return st;
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess)
+        return FP4LIN_ERR_CUDA;
+    float *scratch = nullptr;
+    if ((st = noalloc_scratch(d, &scratch)) != FP4LIN_OK)
+        return st;
+    QuantShape q = make_shape(x, rows, cols, ld_x, codes, scales, 16);
+    const dim3 agrid = amax_grid(q);
+    const int64_t n_partials = (int64_t)agrid.x * agrid.y;
+    if (n_partials > AMAX_MAX_BLOCKS)  // more partial maxima than the array holds
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t s = as_stream(stream);
+    // every partial is written by the amax pass before the quantise pass reads it,
+    // so nothing in the array has to start at zero
+    if (hadamard)
+        nvfp4_amax_kernel<true><<<agrid, QTHREADS, 0, s>>>(q, scratch);
+    else
+        nvfp4_amax_kernel<false><<<agrid, QTHREADS, 0, s>>>(q, scratch);
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    const dim3 grid(quant_grid(q));
+    if (hadamard)
+        nvfp4_quant_kernel<true, true><<<grid, QTHREADS, 0, s>>>(q, g, scratch, (int)n_partials);
+    else
+        nvfp4_quant_kernel<false, true><<<grid, QTHREADS, 0, s>>>(q, g, scratch, (int)n_partials);
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    return launch_padding(q, dev, s);
+}
+
 }  // extern "C"
