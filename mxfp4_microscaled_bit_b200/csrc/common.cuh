@@ -31,6 +31,26 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p)
     return r;
 }
 
+// 32 bytes in one 256-bit load (p must be 32-byte aligned).
+__device__ __forceinline__ void ld_nc_v8(const void *p, uint32_t *r)
+{
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+
+// 32 bytes as one 256-bit load when `wide` (32-byte aligned), else as two 128-bit loads.
+__device__ __forceinline__ void ld_nc_32B(const void *p, bool wide, uint32_t *r)
+{
+    if (wide) {
+        ld_nc_v8(p, r);
+    } else {
+        const uint4 a = ld_nc_v4(p), b = ld_nc_v4(static_cast<const uint8_t *>(p) + 16);
+        r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w;
+        r[4] = b.x; r[5] = b.y; r[6] = b.z; r[7] = b.w;
+    }
+}
+
 __device__ __forceinline__ uint2 ld_nc_v2(const void *p)
 {
     uint2 r;

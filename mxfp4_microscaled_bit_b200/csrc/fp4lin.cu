@@ -245,10 +245,10 @@ int check_quant_args(const void *x, int64_t rows, int64_t cols, int64_t ld_x, co
     return FP4LIN_OK;
 }
 
-// quantiser grid: x = 256-value row segments, y = groups of QROWS rows
+// quantiser grid: x = segments of 32 blocks, y = groups of QROWS rows
 dim3 quant_grid(const QuantShape &q)
 {
-    return dim3((unsigned)((q.chunks_per_row + 31) / 32), (unsigned)((q.rows + QROWS - 1) / QROWS));
+    return dim3((unsigned)((q.blocks_per_row + 31) / 32), (unsigned)((q.rows + QROWS - 1) / QROWS));
 }
 
 // amax pass: the same mapping, grid-strided down to at most AMAX_MAX_BLOCKS CTAs
@@ -279,7 +279,9 @@ QuantShape make_shape(const void *x, int64_t rows, int64_t cols, int64_t ld_x, u
     q.ld = ld_x;
     q.codes = codes;
     q.scales = scales;
-    q.chunks_per_row = cols / 8;
+    q.blocks_per_row = cols / block;
+    // 256-bit loads need every block start 32-byte aligned: the base and the row stride
+    q.wide = (reinterpret_cast<uintptr_t>(x) % 32 == 0) && (ld_x % 16 == 0);
     q.sf_cols = cols / block;
     q.katoms = (q.sf_cols + 3) / 4;
     const int64_t rows_pad = (rows + 127) / 128 * 128;

@@ -9,35 +9,36 @@
 // FP8, NVFP4, MXFP4 i AWQ?".  The rotation is the online activation side of
 // the blockwise Hadamard transform of the MR-GPTQ abstract.
 //
-// Work mapping: one lane owns 8 consecutive bf16 (one 16-byte load).  A
-// 16-value NVFP4 block is a lane pair, a 32-value MXFP4 block a lane quad;
-// the last Hadamard stages and the block maxima cross lanes with shuffles.
-// A warp reads 512 contiguous bytes of one row per load and writes 128
-// contiguous code bytes per store.  Requires cols % 64 == 0, so no block is
-// cut by the end of a row.
+// Work mapping: one lane owns one whole block -- 16 bf16 (32 bytes, one
+// 256-bit load) for NVFP4, 32 bf16 (two loads) for MXFP4 -- so the Hadamard
+// butterflies, the block maximum and the scale arithmetic all stay in the
+// lane's registers and run once per block.  A warp covers 32 consecutive
+// blocks of one row: 1 KB (NVFP4) or 2 KB (MXFP4) of contiguous input and
+// 256 / 512 contiguous code bytes.  Requires cols % 64 == 0.
 #pragma once
 
 #include "common.cuh"
 
 namespace fp4lin {
 
-constexpr int QTHREADS = 256;          // 8 warps
+constexpr int QTHREADS = 256;            // 8 warps
 constexpr int QWARPS = QTHREADS / 32;
-constexpr int QUNROLL = 4;             // rows per warp per pass: four 16-byte loads in flight per lane
-constexpr int QROWS = QWARPS * QUNROLL;  // rows covered by one CTA in one pass (32)
+constexpr int QUNROLL = 4;               // rows per warp per pass: four blocks in flight per lane
+constexpr int QROWS = QWARPS * QUNROLL;  // rows covered by one CTA (32)
 constexpr int AMAX_MAX_BLOCKS = 1024;
 
-// Mapping: CTA (bx, by) covers the 256-value row segment bx of rows
+// Mapping: CTA (bx, by) covers blocks 32*bx .. 32*bx+31 of rows
 // [by*QROWS, by*QROWS + QROWS); warp w handles rows by*QROWS + w + QWARPS*u,
-// lane l the 8 values at column 8*(32*bx + l).  No integer division.
+// lane l block 32*bx + l.  No integer division.
 struct QuantShape {
     const __nv_bfloat16 *x;
     int64_t rows, cols, ld;
     uint8_t *codes, *scales;
-    int64_t chunks_per_row;  // cols / 8
-    int64_t sf_cols;         // cols / block
+    int64_t blocks_per_row;  // cols / block
+    int64_t sf_cols;         // = blocks_per_row
     int64_t katoms;          // ceil(sf_cols / 4)
     int64_t pad_items;       // padding bytes of the scale layout
+    bool wide;               // x and every row start are 32-byte aligned: 256-bit loads
 };
 
 // Byte offset of scale (r, c) in the tensor-core layout (128 x 4 atoms).
@@ -46,64 +47,57 @@ __device__ __forceinline__ int64_t tc_offset(int64_t r, int64_t c, int64_t katom
     return ((r >> 7) * katoms + (c >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (c & 3);
 }
 
-// Butterflies with strides 1, 2, 4 on the lane's 8 consecutive values.
-__device__ __forceinline__ void fwht8(float *v)
+// In-place blockwise Hadamard butterflies on B values, strides 1, 2, 4, ...:
+// the pair (u, w) becomes (u + w, u - w).
+template <int B>
+__device__ __forceinline__ void fwht(float *v)
 {
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1)
+    for (int h = 1; h < B; h <<= 1)
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < B; ++i)
             if ((i & h) == 0) {
-                float u = v[i], w = v[i + h];
+                const float u = v[i], w = v[i + h];
                 v[i] = __fadd_rn(u, w);
                 v[i + h] = __fsub_rn(u, w);
             }
 }
 
-// One butterfly stage across the lane pair (lane, lane ^ mask): the lower
-// lane holds u and keeps u + w, the upper lane holds w and keeps u - w.
-__device__ __forceinline__ void fwht_cross(float *v, int mask, bool upper)
-{
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float o = __shfl_xor_sync(0xffffffffu, v[i], mask);
-        v[i] = upper ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
-    }
-}
-
-__device__ __forceinline__ float abs_max8(const float *v)
+template <int B>
+__device__ __forceinline__ float abs_max(const float *v)
 {
     float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < B; ++i)
         m = fmaxf(m, fabsf(v[i]));
     return m;
 }
 
-// Rotated (when HAD) values of a lane's chunk of a 16-value block.
+// The (rotated, when HAD) values of one NVFP4 block: 16 bf16 in `raw`.
 template <bool HAD>
-__device__ __forceinline__ void nvfp4_lane_values(uint4 raw, bool upper, float *v)
+__device__ __forceinline__ void nvfp4_block_values(const uint32_t *raw, float *v)
 {
-    bf16x8_to_f32(raw, v);
+    bf16x8_to_f32(make_uint4(raw[0], raw[1], raw[2], raw[3]), v);
+    bf16x8_to_f32(make_uint4(raw[4], raw[5], raw[6], raw[7]), v + 8);
     if (HAD) {
-        fwht8(v);
-        fwht_cross(v, 1, upper);
+        fwht<16>(v);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 16; ++j)
             v[j] = __fmul_rn(v[j], 0.25f);  // 1/sqrt(16), exact
     }
 }
 
+// The (rotated, when HAD) values of one MXFP4 block: 32 bf16 in `raw`.
 template <bool HAD>
-__device__ __forceinline__ void mxfp4_lane_values(uint4 raw, int lane, float *v)
+__device__ __forceinline__ void mxfp4_block_values(const uint32_t *raw, float *v)
 {
-    bf16x8_to_f32(raw, v);
-    if (HAD) {
-        fwht8(v);
-        fwht_cross(v, 1, lane & 1);
-        fwht_cross(v, 2, lane & 2);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+    for (int k = 0; k < 4; ++k)
+        bf16x8_to_f32(make_uint4(raw[4 * k], raw[4 * k + 1], raw[4 * k + 2], raw[4 * k + 3]), v + 8 * k);
+    if (HAD) {
+        fwht<32>(v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
             v[j] = __fmul_rn(v[j], 0x1.6a09e6p-3f);  // 1/sqrt(32) rounded to binary32
     }
 }
@@ -127,30 +121,42 @@ __device__ __forceinline__ void zero_scale_padding(const QuantShape &q, int64_t 
     q.scales[tc_offset(r, c, q.katoms)] = 0;
 }
 
+// Zero the padding bytes of a tensor-core scale buffer (launched only when there are any).
+__global__ void __launch_bounds__(QTHREADS) scale_padding_kernel(QuantShape q)
+{
+    for (int64_t j = (int64_t)blockIdx.x * QTHREADS + threadIdx.x; j < q.pad_items; j += (int64_t)gridDim.x * QTHREADS)
+        zero_scale_padding(q, j);
+}
+
 // -------------------------------------------------------------------------
 // Pass 1 of the dynamic tensor scale: per-CTA maxima of |x'| into partials[].
-// Grid-strided over segments (x) and row groups (y); at most AMAX_MAX_BLOCKS CTAs.
+// Grid-strided over block segments (x) and row groups (y); at most
+// AMAX_MAX_BLOCKS CTAs.
 template <bool HAD>
 __global__ void __launch_bounds__(QTHREADS) nvfp4_amax_kernel(QuantShape q, float *partials)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const bool upper = lane & 1;
     float m = 0.0f;
-    for (int64_t seg = blockIdx.x; seg * 32 < q.chunks_per_row; seg += gridDim.x) {
-        const int64_t c8 = seg * 32 + lane;
-        const bool col_ok = c8 < q.chunks_per_row;
+    for (int64_t seg = blockIdx.x; seg * 32 < q.blocks_per_row; seg += gridDim.x) {
+        const int64_t c = seg * 32 + lane;
+        const bool col_ok = c < q.blocks_per_row;
         for (int64_t r0 = (int64_t)blockIdx.y * QROWS; r0 < q.rows; r0 += (int64_t)gridDim.y * QROWS) {
-            uint4 raw[QUNROLL];
+            uint32_t raw[QUNROLL][8];
 #pragma unroll
             for (int u = 0; u < QUNROLL; ++u) {
                 const int64_t r = r0 + warp + QWARPS * u;
-                raw[u] = (col_ok && r < q.rows) ? ld_nc_v4(q.x + r * q.ld + c8 * 8) : make_uint4(0, 0, 0, 0);
+                if (col_ok && r < q.rows)
+                    ld_nc_32B(q.x + r * q.ld + c * 16, q.wide, raw[u]);
+                else
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        raw[u][j] = 0;
             }
 #pragma unroll
             for (int u = 0; u < QUNROLL; ++u) {
-                float v[8];
-                nvfp4_lane_values<HAD>(raw[u], upper, v);
-                m = fmaxf(m, abs_max8(v));
+                float v[16];
+                nvfp4_block_values<HAD>(raw[u], v);
+                m = fmaxf(m, abs_max<16>(v));
             }
         }
     }
@@ -169,15 +175,10 @@ __global__ void __launch_bounds__(QTHREADS) nvfp4_amax_kernel(QuantShape q, floa
     }
 }
 
-// Zero the padding bytes of a tensor-core scale buffer (launched only when there are any).
-__global__ void __launch_bounds__(QTHREADS) scale_padding_kernel(QuantShape q)
-{
-    for (int64_t j = (int64_t)blockIdx.x * QTHREADS + threadIdx.x; j < q.pad_items; j += (int64_t)gridDim.x * QTHREADS)
-        zero_scale_padding(q, j);
-}
-
 // Pass 2: quantise.  DYNAMIC: g = max(partials) / (6*448) (1 if not > 0),
 // written to g_io by CTA (0,0); otherwise g is read from g_io.
+// Per block: t = (amax/6)/g, sf = E4M3(t), d = dec(sf)*g, r = d > 0 ? 1/d : 0,
+// codes = E2M1(x'*r).
 template <bool HAD, bool DYNAMIC>
 __global__ void __launch_bounds__(QTHREADS)
     nvfp4_quant_kernel(QuantShape q, float *g_io, const float *partials, int n_partials)
@@ -185,15 +186,20 @@ __global__ void __launch_bounds__(QTHREADS)
     __shared__ float s_g;
     __shared__ float red[QWARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t c8 = (int64_t)blockIdx.x * 32 + lane;
-    const bool col_ok = c8 < q.chunks_per_row;
+    const int64_t c = (int64_t)blockIdx.x * 32 + lane;
+    const bool col_ok = c < q.blocks_per_row;
     const int64_t r0 = (int64_t)blockIdx.y * QROWS + warp;
     // issue the loads first; the tensor-scale reduction overlaps them
-    uint4 raw[QUNROLL];
+    uint32_t raw[QUNROLL][8];
 #pragma unroll
     for (int u = 0; u < QUNROLL; ++u) {
         const int64_t r = r0 + QWARPS * u;
-        raw[u] = (col_ok && r < q.rows) ? ld_nc_v4(q.x + r * q.ld + c8 * 8) : make_uint4(0, 0, 0, 0);
+        if (col_ok && r < q.rows)
+            ld_nc_32B(q.x + r * q.ld + c * 16, q.wide, raw[u]);
+        else
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                raw[u][j] = 0;
     }
     if (DYNAMIC) {
         float m = 0.0f;
@@ -221,27 +227,23 @@ __global__ void __launch_bounds__(QTHREADS)
     }
     __syncthreads();
     const float g = s_g;
-    const bool upper = lane & 1;
 #pragma unroll
     for (int u = 0; u < QUNROLL; ++u) {
         const int64_t r = r0 + QWARPS * u;
-        float v[8];
-        nvfp4_lane_values<HAD>(raw[u], upper, v);
-        float amax = abs_max8(v);
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        if (!(col_ok && r < q.rows))
+            continue;
+        float v[16];
+        nvfp4_block_values<HAD>(raw[u], v);
+        const float amax = abs_max<16>(v);
         const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
         const uint32_t sf = cvt_e4m3(t);
         const float d = __fmul_rn(e4m3_value(sf), g);
         const float rcp = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 16; ++j)
             v[j] = __fmul_rn(v[j], rcp);
-        const uint32_t packed = pack_e2m1x8(v);
-        if (col_ok && r < q.rows) {
-            *reinterpret_cast<uint32_t *>(q.codes + r * (q.cols / 2) + c8 * 4) = packed;
-            if (!upper)
-                q.scales[tc_offset(r, c8 >> 1, q.katoms)] = (uint8_t)sf;
-        }
+        *reinterpret_cast<uint2 *>(q.codes + r * (q.cols / 2) + c * 8) = make_uint2(pack_e2m1x8(v), pack_e2m1x8(v + 8));
+        q.scales[tc_offset(r, c, q.katoms)] = (uint8_t)sf;
     }
 }
 
@@ -252,34 +254,43 @@ template <bool HAD>
 __global__ void __launch_bounds__(QTHREADS) mxfp4_quant_kernel(QuantShape q)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t c8 = (int64_t)blockIdx.x * 32 + lane;
-    const bool col_ok = c8 < q.chunks_per_row;
+    const int64_t c = (int64_t)blockIdx.x * 32 + lane;
+    const bool col_ok = c < q.blocks_per_row;
     const int64_t r0 = (int64_t)blockIdx.y * QROWS + warp;
-    uint4 raw[QUNROLL];
+    constexpr int U = QUNROLL / 2;  // a block is 64 bytes: two rows in flight per pass
 #pragma unroll
-    for (int u = 0; u < QUNROLL; ++u) {
-        const int64_t r = r0 + QWARPS * u;
-        raw[u] = (col_ok && r < q.rows) ? ld_nc_v4(q.x + r * q.ld + c8 * 8) : make_uint4(0, 0, 0, 0);
-    }
+    for (int half = 0; half < 2; ++half) {
+        uint32_t raw[U][16];
 #pragma unroll
-    for (int u = 0; u < QUNROLL; ++u) {
-        const int64_t r = r0 + QWARPS * u;
-        float v[8];
-        mxfp4_lane_values<HAD>(raw[u], lane, v);
-        float amax = abs_max8(v);
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        const uint32_t E = (__float_as_uint(amax) >> 23) & 0xFFu;
-        const uint32_t byte = E >= 2u ? E - 2u : 0u;
-        const float s = __uint_as_float((254u - byte) << 23);  // 2^(127 - byte)
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = r0 + QWARPS * (u + U * half);
+            if (col_ok && r < q.rows) {
+                const __nv_bfloat16 *p = q.x + r * q.ld + c * 32;
+                ld_nc_32B(p, q.wide, raw[u]);
+                ld_nc_32B(p + 16, q.wide, raw[u] + 8);
+            } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            v[j] = __fmul_rn(v[j], s);
-        const uint32_t packed = pack_e2m1x8(v);
-        if (col_ok && r < q.rows) {
-            *reinterpret_cast<uint32_t *>(q.codes + r * (q.cols / 2) + c8 * 4) = packed;
-            if ((lane & 3) == 0)
-                q.scales[tc_offset(r, c8 >> 2, q.katoms)] = (uint8_t)byte;
+                for (int j = 0; j < 16; ++j)
+                    raw[u][j] = 0;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = r0 + QWARPS * (u + U * half);
+            if (!(col_ok && r < q.rows))
+                continue;
+            float v[32];
+            mxfp4_block_values<HAD>(raw[u], v);
+            const float amax = abs_max<32>(v);
+            const uint32_t E = (__float_as_uint(amax) >> 23) & 0xFFu;
+            const uint32_t byte = E >= 2u ? E - 2u : 0u;
+            const float s = __uint_as_float((254u - byte) << 23);  // 2^(127 - byte)
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                v[j] = __fmul_rn(v[j], s);
+            st_v4(q.codes + r * (q.cols / 2) + c * 16,
+                  make_uint4(pack_e2m1x8(v), pack_e2m1x8(v + 8), pack_e2m1x8(v + 16), pack_e2m1x8(v + 24)));
+            q.scales[tc_offset(r, c, q.katoms)] = (uint8_t)byte;
         }
     }
 }

@@ -150,3 +150,29 @@ def test_mxfp4_extreme_exponents(orc):
     x[3, :] = 1e-39
     check_mxfp4(orc, x)
     check_mxfp4(orc, x, 32)
+
+
+@pytest.mark.parametrize("hadamard", [0, 16])
+def test_nvfp4_narrow_load_path(orc, hadamard):
+    # base only 16-byte aligned and a row stride of 600 elements: no 256-bit loads
+    big = si.student_t_bf16(12, 40, 600)
+    x = big.to(DEV)[:, 8:8 + 512]
+    assert x.data_ptr() % 32 == 16 and x.stride(0) == 600
+    c, s, g = fl.nvfp4_quantize(x, hadamard)
+    status_ok()
+    oc, osl, og = orc.nvfp4_quantize(big[:, 8:8 + 512].contiguous(), hadamard)
+    assert np.array_equal(c.cpu().numpy(), oc)
+    assert np.array_equal(s.cpu().numpy(), orc.tc_scale_layout(osl))
+    assert g.item() == float(og)
+
+
+@pytest.mark.parametrize("hadamard", [0, 32])
+def test_mxfp4_narrow_load_path(orc, hadamard):
+    big = si.student_t_bf16(13, 33, 1048)
+    x = big.to(DEV)[:, 8:8 + 1024]
+    assert x.data_ptr() % 32 == 16
+    c, s = fl.mxfp4_quantize(x, hadamard)
+    status_ok()
+    oc, osl = orc.mxfp4_quantize(big[:, 8:8 + 1024].contiguous(), hadamard)
+    assert np.array_equal(c.cpu().numpy(), oc)
+    assert np.array_equal(s.cpu().numpy(), orc.tc_scale_layout(osl))
