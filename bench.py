@@ -41,6 +41,15 @@ import synthetic_inputs as si  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
+
+# DRAM bytes (read + write) per step for a kernel, from one ncu capture of the current build
+# (profiles/*.md); None where no capture covers the kernel as it stands.
+NCU_TRAFFIC = {
+    "gemm": 287.1e6,          # profiles/gemm_nvfp4_prefill_8192x14336x4096.md, one launch
+    "kv_load_fp8": 5.83e9,    # profiles/kv_load_fp8_8x8x32768x128.md, 1.358 B/element x 2^32 (K and V)
+    "quantize": None,         # the capture covers the quantise pass only, not the amax pass
+    "kv_store": None,
+}
 METRIC = "NVFP4 GEMM TFLOP/s (% dense FP4 peak); quantize/KV GB/s (% of HBM)"
 
 
@@ -445,6 +454,8 @@ def main():
         "quantize": hbm_roof(w.quant_bytes(), q_ms),
         "kv_store": hbm_roof(w.kv_store_bytes(), st_ms),
     }
+    for k, r in rooflines.items():
+        r["traffic"] = NCU_TRAFFIC.get(k)
     rooflines["quantize"]["note"] = "2.5625 B/element (one read of A); the dynamic tensor scale reads A twice"
     rooflines["kv_load_fp8"]["frac_of_8tbs"] = rooflines["kv_load_fp8"]["achieved"] / 8000.0
     shares = {"quantize": q_ms, "gemm": gemm_ms, "kv_store": st_ms, "kv_load_fp8": ld_ms}
