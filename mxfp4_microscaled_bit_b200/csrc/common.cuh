@@ -58,6 +58,14 @@ __device__ __forceinline__ uint2 ld_nc_v2(const void *p)
     return r;
 }
 
+// 32 bytes in one 256-bit store (p must be 32-byte aligned).
+__device__ __forceinline__ void st_v8(void *p, const uint32_t *v)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+                 "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void st_v4(void *p, uint4 v)
 {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)

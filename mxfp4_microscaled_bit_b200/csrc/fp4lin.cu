@@ -469,7 +469,16 @@ int kv_nvfp4_load_fp8(const uint8_t *cache_codes, const uint8_t *cache_scales, c
     const int64_t npair = (L * s.bpr + 1) / 2;
     const int64_t want = std::max<int64_t>(1, (int64_t)dev->sms * 16 / ((int64_t)B * H));
     const int64_t gx = std::min<int64_t>((npair + KV_THREADS - 1) / KV_THREADS, want);
-    kv_load_fp8_kernel<<<dim3((unsigned)gx, (unsigned)(B * H)), KV_THREADS, 0, as_stream(stream)>>>(s);
+    // wide path: whole groups of 8 blocks per slice, every base 32-byte aligned
+    const bool wide = (L * s.bpr) % 8 == 0 && (Lcap * s.bpr) % 8 == 0 && aligned(cache_codes, 32) &&
+                      aligned(cache_scales, 8) && aligned(out_fp8, 32);
+    if (wide) {
+        const int64_t ngrp = L * s.bpr / 8;
+        const int64_t gxw = std::min<int64_t>((ngrp + KV_THREADS - 1) / KV_THREADS, want);
+        kv_load_fp8_wide_kernel<<<dim3((unsigned)gxw, (unsigned)(B * H)), KV_THREADS, 0, as_stream(stream)>>>(s);
+    } else {
+        kv_load_fp8_kernel<<<dim3((unsigned)gx, (unsigned)(B * H)), KV_THREADS, 0, as_stream(stream)>>>(s);
+    }
     return launch_status();
 }
 

@@ -111,6 +111,63 @@ __device__ __forceinline__ uint4 kv_block_fp8(uint2 c, uint32_t sf)
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+// Wide path: a thread takes 8 consecutive blocks -- 64 code bytes (two 256-bit
+// loads), 8 scale bytes (one 64-bit load), 128 FP8 bytes out (four 256-bit
+// stores) -- and keeps two such groups in flight.  Taken when the slice's
+// block count and every base are aligned for it (see kv_load_fp8_wide_ok).
+__device__ __forceinline__ void kv_load_group8(const uint8_t *codes, const uint8_t *scales, uint8_t *out, int64_t grp,
+                                               uint32_t *c, uint2 &sf)
+{
+    ld_nc_v8(codes + grp * 64, c);
+    ld_nc_v8(codes + grp * 64 + 32, c + 8);
+    sf = ld_nc_v2(scales + grp * 8);
+    (void)out;
+}
+
+__global__ void __launch_bounds__(KV_THREADS) kv_load_fp8_wide_kernel(KvLoadShape s)
+{
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        *s.out_scale = __fmul_rn(8.0f, *s.g);
+    const int64_t bh = blockIdx.y;
+    const int64_t nblk = s.L * s.bpr, ngrp = nblk / 8;
+    const uint8_t *codes = s.codes + bh * s.Lcap * s.bpr * 8;
+    const uint8_t *scales = s.scales + bh * s.Lcap * s.bpr;
+    uint8_t *out = s.out + bh * nblk * 16;
+    const int64_t stride = (int64_t)gridDim.x * KV_THREADS;
+    for (int64_t g0 = (int64_t)blockIdx.x * KV_THREADS + threadIdx.x; g0 < ngrp; g0 += 2 * stride) {
+        uint32_t c[2][16];
+        uint2 sf[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t grp = g0 + u * stride;
+            if (grp < ngrp)
+                kv_load_group8(codes, scales, out, grp, c[u], sf[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t grp = g0 + u * stride;
+            if (grp >= ngrp)
+                continue;
+            const uint32_t sw[2] = {sf[u].x, sf[u].y};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {  // two blocks per 256-bit store
+                uint32_t o[8];
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+                    const int blk = 2 * h + b;
+                    const uint4 f = kv_block_fp8(make_uint2(c[u][2 * blk], c[u][2 * blk + 1]),
+                                                 (sw[blk >> 2] >> (8 * (blk & 3))) & 0xFFu);
+                    o[4 * b] = f.x;
+                    o[4 * b + 1] = f.y;
+                    o[4 * b + 2] = f.z;
+                    o[4 * b + 3] = f.w;
+                }
+                st_v8(out + grp * 128 + h * 32, o);
+            }
+        }
+    }
+}
+
 // CTA row y = one (batch, head) slice.  The slice's first L cache rows are
 // contiguous, so block j of the slice sits at code byte 8j and scale byte j
 // and its FP8 output at byte 16j: a flat index, no division.  A thread takes
