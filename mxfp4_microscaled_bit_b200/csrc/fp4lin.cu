@@ -12,6 +12,7 @@
 
 #include "common.cuh"
 #include "gemm_sm100.cuh"
+#include "gemm_sm100_2sm.cuh"
 #include "kv.cuh"
 #include "quantize.cuh"
 
@@ -26,6 +27,7 @@ struct DeviceInfo {
     int status = FP4LIN_OK;
     int sms = 0;
     bool gemm_attr[4] = {false, false, false, false};
+    int pair_clusters[2] = {0, 0};  // resident clusters of the pair kernels (0: not yet queried)
 };
 
 std::mutex g_mutex;
@@ -91,6 +93,23 @@ bool make_code_map(CUtensorMap *m, const uint8_t *codes, int64_t rows, int64_t K
     cuuint32_t estr[2] = {1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over a scale buffer in the tensor-core layout, seen as rows of 256 bytes (half
+// a 512-byte atom each); box = 256 bytes x box_rows, no swizzle, rows past the end read as zero.
+bool make_scale_map(CUtensorMap *m, const uint8_t *scales, int64_t rows, int64_t sf_cols, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return false;
+    const int64_t bytes = (rows + 127) / 128 * 128 * ((sf_cols + 3) / 4 * 4);
+    cuuint64_t dims[2] = {256u, (cuuint64_t)(bytes / 256)};
+    cuuint64_t strides[1] = {256u};
+    cuuint32_t box[2] = {256u, box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(scales), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -191,6 +210,64 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
     return FP4LIN_OK;
 }
 
+// Which kernel runs a GEMM of 256-column tiles that needs no K split: the one-CTA kernel
+// unless FP4LIN_GEMM_KERNEL=pair selects the CTA-pair kernel.  Both give identical results;
+// on the 8192 x 14336 x 4096 prefill product the one-CTA kernel is about 9% faster, since
+// both are limited by the scale copies into TMEM, which the pair does not reduce per SM.
+bool use_pair_kernel(const GemmPlan &pl)
+{
+    if (pl.bn != 256 || pl.splits != 1)
+        return false;
+    const char *e = getenv("FP4LIN_GEMM_KERNEL");
+    return e && strcmp(e, "pair") == 0;
+}
+
+template <class C>
+int launch_gemm_pair(DeviceInfo *dev, int slot, const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a,
+                     const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w, void *y, int64_t M,
+                     int64_t N, int64_t K, int64_t ldy, cudaStream_t st)
+{
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (dev->pair_clusters[slot] == 0) {
+            if (cudaFuncSetAttribute(fp4_gemm_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM_BYTES) != cudaSuccess)
+                return FP4LIN_ERR_CUDA;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3((unsigned)(dev->sms & ~1));
+            cfg.blockDim = dim3(C::THREADS);
+            cfg.dynamicSmemBytes = C::SMEM_BYTES;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, fp4_gemm_pair_kernel<C>, &cfg) != cudaSuccess || n < 1)
+                return FP4LIN_ERR_CUDA;
+            dev->pair_clusters[slot] = n;
+        }
+    }
+    const int64_t sf_cols = C::NV ? K / 16 : K / 32;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB;
+    if (!make_code_map(&tmA, a_codes, M, K, 128) || !make_code_map(&tmB, w_codes, N, K, 128) ||
+        !make_scale_map(&tmSFA, a_scales, M, sf_cols, C::SF_BOX_ROWS) ||
+        !make_scale_map(&tmSFB, w_scales, N, sf_cols, C::SF_BOX_ROWS))
+        return FP4LIN_ERR_CUDA;
+    Gemm2Params p{};
+    p.g_a = g_a;
+    p.g_w = g_w;
+    p.y = reinterpret_cast<__nv_bfloat16 *>(y);
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.ldy = ldy;
+    p.katoms = (sf_cols + 3) / 4;
+    p.num_mt = (int)((M + 255) / 256);
+    p.num_nt = (int)((N + 255) / 256);
+    p.nk = (int)((K + 255) / 256);
+    p.work = (int64_t)p.num_mt * p.num_nt;
+    p.raster = std::max(1, std::min(raster_group(2 * p.num_mt) / 2, p.num_mt));
+    const int64_t clusters = std::min<int64_t>(p.work, dev->pair_clusters[slot]);
+    fp4_gemm_pair_kernel<C><<<(unsigned)(2 * clusters), C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmSFA, tmSFB, p);
+    return launch_status();
+}
+
 int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
                const uint8_t *w_scales, const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
                void *workspace, size_t workspace_bytes, void *stream)
@@ -216,6 +293,13 @@ int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const f
     }
     float *ws = reinterpret_cast<float *>(workspace);
     cudaStream_t s = as_stream(stream);
+    if (use_pair_kernel(pl)) {
+        if (nv)
+            return launch_gemm_pair<Gemm2Cfg<true>>(dev, 0, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N,
+                                                    K, ldy, s);
+        return launch_gemm_pair<Gemm2Cfg<false>>(dev, 1, a_codes, a_scales, nullptr, w_codes, w_scales, nullptr, y,
+                                                 M, N, K, ldy, s);
+    }
     if (nv) {
         if (pl.bn == 256)
             return launch_gemm_cfg<GemmCfg<256, true>>(dev, 0, pl, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y,
