@@ -26,7 +26,7 @@ struct DeviceInfo {
     bool probed = false;
     int status = FP4LIN_OK;
     int sms = 0;
-    bool gemm_attr[4] = {false, false, false, false};
+    bool gemm_attr[6] = {false, false, false, false, false, false};
     int pair_clusters[2] = {0, 0};  // resident clusters of the pair kernels (0: not yet queried)
 };
 
@@ -115,14 +115,50 @@ bool make_scale_map(CUtensorMap *m, const uint8_t *scales, int64_t rows, int64_t
 
 // ------------------------------------------------------------------ GEMM planning
 struct GemmPlan {
+    bool swap;  // decode form: the MMA runs y^T = W A^T over 128-row weight tiles
     int bn;
     int splits, kps, nk, num_mt, num_nt;
     int64_t ldw;
     size_t ws_bytes;
 };
 
+// Decode form (M <= 16): tiles of 128 weight rows, K split s ways.  s minimises the k-tiles the
+// busiest CTA streams, ceil(tiles*s / sms) * ceil(nk / s), plus, for s > 1, the partial sums'
+// round trip through HBM and the reduction launch, both counted in the same k-tile units
+// (one unit = one 128 x 256 weight tile with its scales, ~18 KB).
+GemmPlan plan_decode(int64_t M, int64_t N, int64_t K, int sms)
+{
+    GemmPlan p{};
+    p.swap = true;
+    p.bn = 16;
+    p.num_mt = (int)((N + 127) / 128);
+    p.num_nt = 1;
+    p.nk = (int)((K + 255) / 256);
+    p.ldw = (N + 3) / 4 * 4;
+    double best = 1e300;
+    for (int s = 1; s <= std::min(p.nk, 16); ++s) {
+        const int kps = (p.nk + s - 1) / s;
+        const int eff = (p.nk + kps - 1) / kps;  // splits actually used
+        if (eff != s)
+            continue;
+        const int64_t waves = ((int64_t)p.num_mt * s + sms - 1) / sms;
+        double cost = (double)(waves * kps);
+        if (s > 1)
+            cost += 4.0 + 2.0 * s * (double)M * (double)p.ldw * 4.0 / ((double)sms * 18432.0);
+        if (cost < best) {
+            best = cost;
+            p.splits = s;
+            p.kps = kps;
+        }
+    }
+    p.ws_bytes = p.splits > 1 ? (size_t)p.splits * (size_t)M * (size_t)p.ldw * sizeof(float) : 0;
+    return p;
+}
+
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms)
 {
+    if (M <= 16)
+        return plan_decode(M, N, K, sms);
     GemmPlan p{};
     p.bn = (M > 128 && N > 128) ? 256 : 64;
     p.num_mt = (int)((M + 127) / 128);
@@ -199,9 +235,10 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
     if (launch_status() != FP4LIN_OK)
         return FP4LIN_ERR_CUDA;
     if (pl.splits > 1) {
-        const int64_t items = M * ((N + 3) / 4);
+        const int64_t rM = C::SWAP ? N : M, rN = C::SWAP ? M : N;  // the output's shape
+        const int64_t items = rM * ((rN + 3) / 4);
         const int rgrid = (int)std::min<int64_t>((items + 255) / 256, (int64_t)dev->sms * 8);
-        splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(ws, pl.splits, M, N, pl.ldw, C::NV ? g_a : nullptr,
+        splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(ws, pl.splits, rM, rN, pl.ldw, C::NV ? g_a : nullptr,
                                                     C::NV ? g_w : nullptr, reinterpret_cast<__nv_bfloat16 *>(y),
                                                     ldy);
         if (launch_status() != FP4LIN_OK)
@@ -293,6 +330,13 @@ int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const f
     }
     float *ws = reinterpret_cast<float *>(workspace);
     cudaStream_t s = as_stream(stream);
+    if (pl.swap) {  // the weights take the MMA's M side: operands and shapes swap places
+        if (nv)
+            return launch_gemm_cfg<GemmCfg<16, true, true>>(dev, 4, pl, w_codes, w_scales, g_w, a_codes, a_scales,
+                                                            g_a, y, N, M, K, ldy, ws, s);
+        return launch_gemm_cfg<GemmCfg<16, false, true>>(dev, 5, pl, w_codes, w_scales, nullptr, a_codes, a_scales,
+                                                         nullptr, y, N, M, K, ldy, ws, s);
+    }
     if (use_pair_kernel(pl)) {
         if (nv)
             return launch_gemm_pair<Gemm2Cfg<true>>(dev, 0, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N,

@@ -184,6 +184,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v)
         v[i] = __uint_as_float(r[i]);
 }
 
+// 8 consecutive accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v)
+{
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        v[i] = __uint_as_float(r[i]);
+}
+
 // Shared-memory matrix descriptor, K-major with the 128-byte swizzle: rows of
 // 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), version 1.
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
@@ -200,10 +214,14 @@ __device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr)
 }
 
 // ------------------------------------------------------------------ configuration
-template <int BN_, bool NV_>
+// SWAP: the MMA computes y^T = W A^T -- its M operand is W (128 rows per tile), its N
+// operand the few activation rows (BN = 16) -- and the epilogue writes y transposed.  For
+// decode-sized M every tile then streams 128 weight rows instead of padding M to 128.
+template <int BN_, bool NV_, bool SWAP_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool NV = NV_;                       // NVFP4 (16-blocks, E4M3) or MXFP4 (32-blocks, E8M0)
+    static constexpr bool SWAP = SWAP_;
     static constexpr int BM = 128;
     static constexpr int BK = 256;                        // elements per stage (128 code bytes per row)
     static constexpr int MMA_K = 64;
@@ -232,6 +250,8 @@ struct GemmCfg {
     static_assert(TMEM_USED <= 512, "TMEM overflow");
     static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
     static_assert(STAGES >= 2, "pipeline too shallow");
+    static_assert(!SWAP || BN == 16, "the swapped form serves at most 16 activation rows");
+    static_assert(SWAP || COLS_PER_WARP % 32 == 0, "epilogue loads 32 columns at a time");
 };
 
 struct GemmParams {
@@ -445,11 +465,33 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tc_fence_after();
             float v[C::COLS_PER_WARP];
             const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + acc * C::BN + half * C::COLS_PER_WARP;
+            if constexpr (C::SWAP) {
+                tmem_ld8(taddr, v);
+            } else {
 #pragma unroll
-            for (int c = 0; c < C::COLS_PER_WARP; c += 32)
-                tmem_ld32(taddr + c, v + c);
+                for (int c = 0; c < C::COLS_PER_WARP; c += 32)
+                    tmem_ld32(taddr + c, v + c);
+            }
             tc_fence_before();
             mbar_arrive(&acc_empty[acc]);  // accumulator free: the next tile's MMAs may start
+
+            if constexpr (C::SWAP) {
+                // accumulator row = weight row n, column = activation row m: y[m, n]
+                const int64_t n = (int64_t)mt * C::BM + quad * 32 + lane;
+                if (n < p.M) {
+#pragma unroll
+                    for (int c = 0; c < C::COLS_PER_WARP; ++c) {
+                        const int64_t m = (int64_t)nt * C::BN + half * C::COLS_PER_WARP + c;
+                        if (m < p.N) {
+                            if (p.splits == 1)
+                                p.y[m * p.ldy + n] = __float2bfloat16_rn(__fmul_rn(v[c], gg));
+                            else
+                                p.ws[((int64_t)sp * p.N + m) * p.ldw + n] = v[c];
+                        }
+                    }
+                }
+                continue;
+            }
 
             const int64_t m = (int64_t)mt * C::BM + quad * 32 + lane;
             const int64_t n0 = (int64_t)nt * C::BN + half * C::COLS_PER_WARP;
