@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
                 "oracle_nvfp4_tensor_scale": (ctypes.c_float, [u16p, i64, i64, i64, ctypes.c_int]),
                 "oracle_nvfp4_quantize": (None, [u16p, i64, i64, i64, ctypes.c_int, ctypes.c_float, u8p, u8p]),
                 "oracle_mxfp4_quantize": (None, [u16p, i64, i64, i64, ctypes.c_int, u8p, u8p]),
+                "oracle_nvfp4_quantize_mse": (None, [u16p, i64, i64, i64, ctypes.c_int, ctypes.c_float, u8p, u8p]),
+                "oracle_mxfp4_quantize_nearest": (None, [u16p, i64, i64, i64, ctypes.c_int, u8p, u8p]),
                 "oracle_tc_scale_bytes": (i64, [i64, i64]),
                 "oracle_tc_scale_layout": (None, [u8p, i64, i64, u8p]),
                 "oracle_dequant": (None, [u8p, u8p, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_double, f64p]),
@@ -173,14 +175,29 @@ def nvfp4_quantize(x, hadamard: int = 0, g=None):
     return codes, sf, np.float32(g)
 
 
-def mxfp4_quantize(x, hadamard: int = 0):
-    """-> (codes uint8 [rows, cols/2], sf uint8 [rows, cols/32] row-major E8M0)."""
+def nvfp4_quantize_mse(x, hadamard: int = 0, g=None):
+    """NVFP4 with the MSE-optimal block scale (reading R9): brute force over all 127
+    non-negative finite E4M3 scales per block.  Same outputs as nvfp4_quantize."""
+    xb = _bits(x)
+    rows, cols = xb.shape
+    if g is None:
+        g = nvfp4_tensor_scale(xb, hadamard)
+    codes = np.zeros((rows, cols // 2), dtype=np.uint8)
+    sf = np.zeros((rows, cols // 16), dtype=np.uint8)
+    lib().oracle_nvfp4_quantize_mse(_p(xb, ctypes.c_uint16), rows, cols, cols, hadamard, float(g),
+                                    _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8))
+    return codes, sf, np.float32(g)
+
+
+def mxfp4_quantize(x, hadamard: int = 0, nearest: bool = False):
+    """-> (codes uint8 [rows, cols/2], sf uint8 [rows, cols/32] row-major E8M0).
+    nearest: the nearest-power-of-two scale (reading R10) instead of the OCP rule (R4)."""
     xb = _bits(x)
     rows, cols = xb.shape
     codes = np.zeros((rows, cols // 2), dtype=np.uint8)
     sf = np.zeros((rows, cols // 32), dtype=np.uint8)
-    lib().oracle_mxfp4_quantize(_p(xb, ctypes.c_uint16), rows, cols, cols, hadamard,
-                                _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8))
+    fn = lib().oracle_mxfp4_quantize_nearest if nearest else lib().oracle_mxfp4_quantize
+    fn(_p(xb, ctypes.c_uint16), rows, cols, cols, hadamard, _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8))
     return codes, sf
 
 

@@ -40,6 +40,16 @@
  *      ordered row-tile-major; in an atom, byte (r%32)*16 + ((r%128)/32)*4 + c%4.
  *   R8 KV: static per-tensor g; dequantised FP8 = E4M3(e2m1 * dec(sf) / 8),
  *      attention-side scale 8*g.
+ *   R9 NVFP4 "MSE-optimal" block scale ([FP4-BW]: the scale minimises the mean
+ *      squared error over the block's 16 values): every non-negative finite
+ *      E4M3 code c = 0..126 is tried with d = RN32(dec(c)*g), r = RN32(1/d)
+ *      (0 when d = 0), q_i = E2M1(RN32(x_i*r)); its error is the binary32 sum,
+ *      in order i = 0..15, of RN32(RN32(x_i - RN32(e2m1(q_i)*d))^2); the
+ *      smallest error wins, ties to the smaller code.  g is R3's.
+ *   R10 MXFP4 "nearest power of two" ([FP4-BW]: the scale is rounded to the
+ *      nearest power of two): the ideal scale amax/6 is rounded to the nearer
+ *      of the two powers of two around it, by value, ties upward.  With
+ *      e = floor(log2 amax) that is X = e-2 when amax >= 1.125*2^e, else e-3.
  */
 #include <math.h>
 #include <stdint.h>
@@ -247,6 +257,52 @@ static uint8_t nvfp4_block(const float *x, float g, uint8_t *codes)
     return sf;
 }
 
+/* One 16-value block with the MSE-optimal E4M3 block scale ([FP4-BW]: the
+ * scaling algorithm picks the factor with the least mean squared error over
+ * the block's 16 values; reading R9 for the candidate set, the arithmetic and
+ * the tie rule).  Every candidate is tried: a brute-force search. */
+static uint8_t nvfp4_block_mse(const float *x, float g, uint8_t *codes)
+{
+    int best = -1;
+    float best_err = 0.0f;
+    uint8_t q[16];
+    for (int c = 0; c <= 126; ++c) {
+        float d = (float)oracle_e4m3_decode((uint8_t)c) * g;
+        float rcp = (d > 0.0f) ? 1.0f / d : 0.0f;
+        float err = 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            q[i] = oracle_e2m1_encode(x[i] * rcp);
+            float t = (float)oracle_e2m1_decode(q[i]) * d;
+            float diff = x[i] - t;
+            err = err + diff * diff;
+        }
+        if (best < 0 || err < best_err) {
+            best = c;
+            best_err = err;
+            memcpy(codes, q, 16);
+        }
+    }
+    return (uint8_t)best;
+}
+
+/* NVFP4 quantisation with the MSE-optimal block scales (R9); same layouts and
+ * tensor scale as oracle_nvfp4_quantize. */
+EXPORT void oracle_nvfp4_quantize_mse(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                      int hadamard, float g, uint8_t *codes, uint8_t *sf)
+{
+    int64_t nb = cols / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < nb; ++k) {
+            float blk[16];
+            uint8_t c[16];
+            load_block(x, ld, r, k, 16, hadamard, blk);
+            sf[r * nb + k] = nvfp4_block_mse(blk, g, c);
+            for (int j = 0; j < 8; ++j)
+                codes[r * (cols / 2) + k * 8 + j] = (uint8_t)(c[2 * j] | (c[2 * j + 1] << 4));
+        }
+}
+
 /* NVFP4 quantisation of a bf16 [rows, cols] matrix (row stride ld elements).
  * codes: [rows, cols/2] packed (R6).  sf: [rows, cols/16] row-major E4M3. */
 EXPORT void oracle_nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
@@ -268,8 +324,9 @@ EXPORT void oracle_nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols,
 
 /* One 32-value block with a power-of-two E8M0 scale ([FP4-BW]: MXFP4 from the
  * OCP Microscaling spec, E8M0 scaling, 32 values per block; [PL]: OCP,
- * 32-value blocks, power-of-two E8M0 scale; reading R4 for the exponent rule). */
-static uint8_t mxfp4_block(const float *x, uint8_t *codes)
+ * 32-value blocks, power-of-two E8M0 scale; reading R4 for the exponent rule,
+ * or R10 when `nearest`). */
+static uint8_t mxfp4_block(const float *x, uint8_t *codes, int nearest)
 {
     float amax = 0.0f;
     for (int i = 0; i < 32; ++i)
@@ -282,6 +339,8 @@ static uint8_t mxfp4_block(const float *x, uint8_t *codes)
         int e;
         frexp((double)amax, &e);    /* amax = f * 2^e, f in [0.5, 1): floor(log2 amax) = e - 1 */
         int X = (e - 1) - 2;        /* 2 = exponent of E2M1's largest power of two, 4 */
+        if (nearest && (double)amax < 1.125 * ldexp(1.0, e - 1))
+            X -= 1;                 /* amax/6 < 1.5 * 2^(X-1): the lower power of two is nearer */
         byte = X + 127;
         if (byte < 0)
             byte = 0;
@@ -294,9 +353,10 @@ static uint8_t mxfp4_block(const float *x, uint8_t *codes)
     return (uint8_t)byte;
 }
 
-/* MXFP4 quantisation.  codes: [rows, cols/2]; sf: [rows, cols/32] row-major E8M0. */
-EXPORT void oracle_mxfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
-                                  int hadamard, uint8_t *codes, uint8_t *sf)
+/* MXFP4 quantisation.  codes: [rows, cols/2]; sf: [rows, cols/32] row-major E8M0.
+ * nearest = 0: the OCP exponent rule (R4); 1: the nearest power of two (R10). */
+static void mxfp4_quantize_rule(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                int hadamard, uint8_t *codes, uint8_t *sf, int nearest)
 {
     int64_t nb = cols / 32;
     for (int64_t r = 0; r < rows; ++r)
@@ -304,10 +364,22 @@ EXPORT void oracle_mxfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols,
             float blk[32];
             uint8_t c[32];
             load_block(x, ld, r, k, 32, hadamard, blk);
-            sf[r * nb + k] = mxfp4_block(blk, c);
+            sf[r * nb + k] = mxfp4_block(blk, c, nearest);
             for (int j = 0; j < 16; ++j)
                 codes[r * (cols / 2) + k * 16 + j] = (uint8_t)(c[2 * j] | (c[2 * j + 1] << 4));
         }
+}
+
+EXPORT void oracle_mxfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                  int hadamard, uint8_t *codes, uint8_t *sf)
+{
+    mxfp4_quantize_rule(x, rows, cols, ld, hadamard, codes, sf, 0);
+}
+
+EXPORT void oracle_mxfp4_quantize_nearest(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                          int hadamard, uint8_t *codes, uint8_t *sf)
+{
+    mxfp4_quantize_rule(x, rows, cols, ld, hadamard, codes, sf, 1);
 }
 
 /* ------------------------------------------------------------------ scale layout (R7) */
