@@ -208,6 +208,37 @@ int nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld
                            int hadamard, float *g, uint8_t *codes, uint8_t *scales,
                            void *stream);
 
+/*
+ * NVFP4 quantisation with the block scale that minimises the block's squared
+ * error (page "FP4 auf Blackwell: Was NVFP4 fuer lokale KI wirklich aendert",
+ * section "Was NVFP4 von frueheren 4-Bit-Formaten unterscheidet": the scaling
+ * algorithm picks the factor with the least mean squared error over the 16
+ * values of a block).  Meant for weights, offline.  The tensor scale g is
+ * nvfp4_quantize's (amax / 2688, computed or given); for every 16-value block
+ * all 127 non-negative finite E4M3 codes c are tried: d = RN32(dec(c) * g),
+ * r = RN32(1/d) (0 when d = 0), q_i = E2M1(RN32(x_i * r)), error = binary32
+ * sum in order i = 0..15 of RN32(RN32(x_i - RN32(e2m1(q_i) * d))^2); the least
+ * error wins, ties to the smaller code.  Tensors whose amax is below ~1e-32
+ * (where 1/d overflows for small codes) are outside the specified range.
+ * Arguments, layouts, workspace and errors exactly as nvfp4_quantize.
+ */
+int nvfp4_quantize_mse(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                       int hadamard, int compute_global_scale, float *g,
+                       uint8_t *codes, uint8_t *scales,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * MXFP4 quantisation with the E8M0 scale rounded to the nearest power of two
+ * (same page and section: E8M0 rounds the scale factor to the nearest power
+ * of two): the ideal scale amax/6 goes to the nearer of the two powers of two
+ * around it, by value, ties upward.  With e = floor(log2 amax) that is
+ * X = e - 2 when amax >= 1.125 * 2^e, else X = e - 3 (values then saturate at
+ * 6); byte = clamp(X + 127, 0, 254), codes = E2M1 of x' * 2^-X.
+ * Arguments, layouts and errors exactly as mxfp4_quantize.
+ */
+int mxfp4_quantize_nearest(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                           int hadamard, uint8_t *codes, uint8_t *scales, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -48,6 +48,8 @@ EXPORTS = {
     "fp4lin_device_status": (_int, [_vp]),
     "fp4lin_convert_selftest": (_int, [_vp, _vp, _vp, _i64, _vp]),
     "nvfp4_quantize_noalloc": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
+    "nvfp4_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mxfp4_quantize_nearest": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp]),
 }
 
 _lock = threading.Lock()
@@ -109,12 +111,14 @@ def device_status(stream=None) -> int:
 # ------------------------------------------------------------------ quantisers
 def nvfp4_quantize(x: torch.Tensor, hadamard: int = 0, g: torch.Tensor | None = None, *,
                    compute_global_scale: bool | None = None, codes: torch.Tensor | None = None,
-                   scales: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+                   scales: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None,
+                   mse: bool = False):
     """NVFP4-quantise bf16 x [rows, cols] (row stride x.stride(0)).
 
     By default the FP32 tensor scale is computed when g is None (returned as a new 1-element
     device tensor) and used as given otherwise.  compute_global_scale=True with a g tensor
-    writes the computed scale into that tensor.
+    writes the computed scale into that tensor.  mse=True chooses every block scale by the
+    least squared error over all E4M3 scales (nvfp4_quantize_mse) instead of amax/6.
     Returns (codes uint8 [rows, cols/2], scales uint8 [scale_bytes], g).
     """
     rows, cols = x.shape
@@ -131,7 +135,8 @@ def nvfp4_quantize(x: torch.Tensor, hadamard: int = 0, g: torch.Tensor | None = 
     if scales is None:
         scales = torch.empty(scale_bytes(rows, cols // 16), dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check("nvfp4_quantize", lib().nvfp4_quantize(
+    name = "nvfp4_quantize_mse" if mse else "nvfp4_quantize"
+    _check(name, getattr(lib(), name)(
         _ptr(x), rows, cols, x.stride(0), hadamard, 1 if dynamic else 0, _ptr(g), _ptr(codes), _ptr(scales),
         _ptr(workspace), ws_bytes, _stream(stream)))
     return codes, scales, g
@@ -148,15 +153,17 @@ def nvfp4_quantize_noalloc(x: torch.Tensor, hadamard: int, g: torch.Tensor, code
 
 
 def mxfp4_quantize(x: torch.Tensor, hadamard: int = 0, *, codes: torch.Tensor | None = None,
-                   scales: torch.Tensor | None = None, stream=None):
-    """MXFP4-quantise bf16 x [rows, cols] -> (codes uint8 [rows, cols/2], scales uint8 [scale_bytes])."""
+                   scales: torch.Tensor | None = None, stream=None, nearest: bool = False):
+    """MXFP4-quantise bf16 x [rows, cols] -> (codes uint8 [rows, cols/2], scales uint8 [scale_bytes]).
+    nearest=True rounds each scale to the nearest power of two (mxfp4_quantize_nearest)."""
     rows, cols = x.shape
     if codes is None:
         codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(scale_bytes(rows, cols // 32), dtype=torch.uint8, device=x.device)
-    _check("mxfp4_quantize", lib().mxfp4_quantize(_ptr(x), rows, cols, x.stride(0), hadamard, _ptr(codes),
-                                                  _ptr(scales), _stream(stream)))
+    name = "mxfp4_quantize_nearest" if nearest else "mxfp4_quantize"
+    _check(name, getattr(lib(), name)(_ptr(x), rows, cols, x.stride(0), hadamard, _ptr(codes), _ptr(scales),
+                                      _stream(stream)))
     return codes, scales
 
 

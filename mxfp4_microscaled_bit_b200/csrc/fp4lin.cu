@@ -15,6 +15,7 @@
 #include "gemm_sm100_2sm.cuh"
 #include "kv.cuh"
 #include "quantize.cuh"
+#include "scale_search.cuh"
 
 using namespace fp4lin;
 
@@ -495,8 +496,58 @@ int nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
     return launch_padding(q, dev, s);
 }
 
-int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard, uint8_t *codes,
-                   uint8_t *scales, void *stream)
+int nvfp4_quantize_mse(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard,
+                       int compute_global_scale, float *g, uint8_t *codes, uint8_t *scales, void *workspace,
+                       size_t workspace_bytes, void *stream)
+{
+    int st = check_quant_args(x, rows, cols, ld_x, codes, scales);
+    if (st != FP4LIN_OK)
+        return st;
+    if (!g || (hadamard != 0 && hadamard != 16) || (compute_global_scale != 0 && compute_global_scale != 1))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (!aligned(g, 4))
+        return FP4LIN_ERR_MISALIGNED;
+    if (compute_global_scale) {
+        if (!workspace || workspace_bytes < AMAX_MAX_BLOCKS * sizeof(float))
+            return FP4LIN_ERR_WORKSPACE;
+        if (!aligned(workspace, 4))
+            return FP4LIN_ERR_MISALIGNED;
+    }
+    DeviceInfo *dev = nullptr;
+    if ((st = current_device(&dev)) != FP4LIN_OK)
+        return st;
+    QuantShape q = make_shape(x, rows, cols, ld_x, codes, scales, 16);
+    cudaStream_t s = as_stream(stream);
+    float *partials = reinterpret_cast<float *>(workspace);
+    int n_partials = 0;
+    if (compute_global_scale) {
+        const dim3 agrid = amax_grid(q);
+        n_partials = (int)(agrid.x * agrid.y);
+        if (hadamard)
+            nvfp4_amax_kernel<true><<<agrid, QTHREADS, 0, s>>>(q, partials);
+        else
+            nvfp4_amax_kernel<false><<<agrid, QTHREADS, 0, s>>>(q, partials);
+        if (launch_status() != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+    }
+    // one warp per block, grid-strided over the blocks
+    const int64_t nblocks = rows * (cols / 16);
+    const unsigned grid = (unsigned)std::min<int64_t>((nblocks + QWARPS - 1) / QWARPS, (int64_t)dev->sms * 16);
+    if (hadamard && compute_global_scale)
+        nvfp4_quant_mse_kernel<true, true><<<grid, QTHREADS, 0, s>>>(q, g, partials, n_partials);
+    else if (hadamard)
+        nvfp4_quant_mse_kernel<true, false><<<grid, QTHREADS, 0, s>>>(q, g, partials, 0);
+    else if (compute_global_scale)
+        nvfp4_quant_mse_kernel<false, true><<<grid, QTHREADS, 0, s>>>(q, g, partials, n_partials);
+    else
+        nvfp4_quant_mse_kernel<false, false><<<grid, QTHREADS, 0, s>>>(q, g, partials, 0);
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    return launch_padding(q, dev, s);
+}
+
+static int mxfp4_quantize_rule(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard,
+                               uint8_t *codes, uint8_t *scales, void *stream, bool nearest)
 {
     int st = check_quant_args(x, rows, cols, ld_x, codes, scales);
     if (st != FP4LIN_OK)
@@ -509,13 +560,29 @@ int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
     QuantShape q = make_shape(x, rows, cols, ld_x, codes, scales, 32);
     cudaStream_t s = as_stream(stream);
     const dim3 grid(quant_grid(q));
-    if (hadamard)
-        mxfp4_quant_kernel<true><<<grid, QTHREADS, 0, s>>>(q);
+    if (hadamard && nearest)
+        mxfp4_quant_kernel<true, true><<<grid, QTHREADS, 0, s>>>(q);
+    else if (hadamard)
+        mxfp4_quant_kernel<true, false><<<grid, QTHREADS, 0, s>>>(q);
+    else if (nearest)
+        mxfp4_quant_kernel<false, true><<<grid, QTHREADS, 0, s>>>(q);
     else
-        mxfp4_quant_kernel<false><<<grid, QTHREADS, 0, s>>>(q);
+        mxfp4_quant_kernel<false, false><<<grid, QTHREADS, 0, s>>>(q);
     if (launch_status() != FP4LIN_OK)
         return FP4LIN_ERR_CUDA;
     return launch_padding(q, dev, s);
+}
+
+int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard, uint8_t *codes,
+                   uint8_t *scales, void *stream)
+{
+    return mxfp4_quantize_rule(x, rows, cols, ld_x, hadamard, codes, scales, stream, false);
+}
+
+int mxfp4_quantize_nearest(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int hadamard, uint8_t *codes,
+                           uint8_t *scales, void *stream)
+{
+    return mxfp4_quantize_rule(x, rows, cols, ld_x, hadamard, codes, scales, stream, true);
 }
 
 int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,

@@ -250,7 +250,12 @@ __global__ void __launch_bounds__(QTHREADS)
 // MXFP4: E8M0 byte = max(E - 2, 0) where E is the biased binary32 exponent
 // of the block maximum (= clamp(floor(log2 amax) - 2 + 127, 0, 254) for
 // finite inputs); elements are scaled by 2^(127 - byte), an exact product.
-template <bool HAD>
+// NEAREST: the scale amax/6 rounded to the nearer power of two by value, ties
+// upward (page "FP4 auf Blackwell", section "Was NVFP4 von frueheren
+// 4-Bit-Formaten unterscheidet": E8M0 rounds the scale to the nearest power of
+// two): one step lower than the rule above exactly when amax < 1.125 * 2^(E-127),
+// i.e. when the stored mantissa is below 2^20.
+template <bool HAD, bool NEAREST = false>
 __global__ void __launch_bounds__(QTHREADS) mxfp4_quant_kernel(QuantShape q)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -282,8 +287,10 @@ __global__ void __launch_bounds__(QTHREADS) mxfp4_quant_kernel(QuantShape q)
             float v[32];
             mxfp4_block_values<HAD>(raw[u], v);
             const float amax = abs_max<32>(v);
-            const uint32_t E = (__float_as_uint(amax) >> 23) & 0xFFu;
-            const uint32_t byte = E >= 2u ? E - 2u : 0u;
+            const uint32_t bits = __float_as_uint(amax);
+            const uint32_t E = (bits >> 23) & 0xFFu;
+            const uint32_t lower = (NEAREST && (bits & 0x7FFFFFu) < 0x100000u) ? 1u : 0u;
+            const uint32_t byte = E >= 2u + lower ? E - 2u - lower : 0u;
             const float s = __uint_as_float((254u - byte) << 23);  // 2^(127 - byte)
 #pragma unroll
             for (int j = 0; j < 32; ++j)

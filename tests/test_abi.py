@@ -23,7 +23,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported():
     names = header_functions()
-    assert len(names) == 13, names
+    assert len(names) == 15, names
     L = fl.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -50,11 +50,15 @@ def test_sizes():
     assert L.fp4lin_gemm_workspace_bytes(16, 4096, 4096) > 0
 
 
-def q(x=P, rows=16, cols=128, ld=128, had=0, dyn=0, g=P, codes=P, scales=P, ws=P, wsb=4096):
-    return fl.lib().nvfp4_quantize(x, rows, cols, ld, had, dyn, g, codes, scales, ws, wsb, None)
+def quant_call(x=P, rows=16, cols=128, ld=128, had=0, dyn=0, g=P, codes=P, scales=P, ws=P, wsb=4096, fn="nvfp4_quantize"):
+    return getattr(fl.lib(), fn)(x, rows, cols, ld, had, dyn, g, codes, scales, ws, wsb, None)
 
 
-def test_nvfp4_quantize_argument_checks():
+@pytest.mark.parametrize("fn", ["nvfp4_quantize", "nvfp4_quantize_mse"])
+def test_nvfp4_quantize_argument_checks(fn):
+    def q(**kw):
+        return quant_call(fn=fn, **kw)
+
     assert q(x=None) == INVALID
     assert q(codes=None) == INVALID
     assert q(g=None) == INVALID
@@ -70,11 +74,12 @@ def test_nvfp4_quantize_argument_checks():
     assert q(dyn=1, wsb=100) == WORKSPACE
 
 
-def test_mxfp4_quantize_argument_checks():
-    L = fl.lib()
-    assert L.mxfp4_quantize(P, 4, 128, 128, 16, P, P, None) == INVALID
-    assert L.mxfp4_quantize(P, 4, 96, 96, 0, P, P, None) == SHAPE
-    assert L.mxfp4_quantize(P + 2, 4, 128, 128, 0, P, P, None) == MISALIGNED
+@pytest.mark.parametrize("fn", ["mxfp4_quantize", "mxfp4_quantize_nearest"])
+def test_mxfp4_quantize_argument_checks(fn):
+    f = getattr(fl.lib(), fn)
+    assert f(P, 4, 128, 128, 16, P, P, None) == INVALID
+    assert f(P, 4, 96, 96, 0, P, P, None) == SHAPE
+    assert f(P + 2, 4, 128, 128, 0, P, P, None) == MISALIGNED
 
 
 def g(M=16, N=64, K=128, ldy=64, a=P, y=P, ga=P):
