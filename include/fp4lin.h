@@ -209,6 +209,27 @@ int nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld
                            void *stream);
 
 /*
+ * nvfp4_gemm whose output is also NVFP4-quantised for the next layer, inside the
+ * GEMM's epilogue (or its split-K reduction), so a chain of layers need not
+ * write and re-read bf16.  The output is first rounded to bf16 exactly as
+ * nvfp4_gemm rounds it; then each 16-value block of each output row is rotated
+ * by H_16/4 when hadamard = 16 and encoded as nvfp4_quantize does with the
+ * STATIC tensor scale *g_y: the codes and scales equal those of
+ * nvfp4_quantize(y, hadamard, *g_y) applied to the bf16 y, bit for bit.
+ *   y: bf16 [M, N] with row stride ldy, or NULL (then only the codes are written);
+ *   y_codes [M, N/2]; y_scales tensor-core layout of [M, N/16] (padding zeroed).
+ * Shapes as nvfp4_gemm and N a multiple of 64 (FP4LIN_ERR_UNSUPPORTED_SHAPE).
+ * g_y device float (4-byte aligned); y_codes, y_scales 16-byte aligned.
+ * Errors as nvfp4_gemm; hadamard not 0 or 16, or a null g_y, y_codes or
+ * y_scales, give FP4LIN_ERR_INVALID_ARGUMENT.
+ */
+int nvfp4_gemm_quant(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a,
+                     const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w,
+                     void *y, int64_t ldy, int hadamard, const float *g_y,
+                     uint8_t *y_codes, uint8_t *y_scales, int64_t M, int64_t N, int64_t K,
+                     void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * NVFP4 quantisation with the block scale that minimises the block's squared
  * error (page "FP4 auf Blackwell: Was NVFP4 fuer lokale KI wirklich aendert",
  * section "Was NVFP4 von frueheren 4-Bit-Formaten unterscheidet": the scaling

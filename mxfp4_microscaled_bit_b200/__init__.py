@@ -50,6 +50,8 @@ EXPORTS = {
     "nvfp4_quantize_noalloc": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_quantize_nearest": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp]),
+    "nvfp4_gemm_quant": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _vp, _vp, _vp, _i64, _i64, _i64,
+                                _vp, _sz, _vp]),
 }
 
 _lock = threading.Lock()
@@ -190,6 +192,26 @@ def nvfp4_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, *, out=None, work
     _check("nvfp4_gemm", lib().nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(g_a), _ptr(w_codes), _ptr(w_scales),
                                           _ptr(g_w), _ptr(y), M, N, K, y.stride(0), _ptr(ws), wsb, _stream(stream)))
     return y
+
+
+def nvfp4_gemm_quant(a_codes, a_scales, g_a, w_codes, w_scales, g_w, g_y, *, hadamard: int = 0,
+                     out=None, write_y: bool = True, y_codes=None, y_scales=None, workspace=None, stream=None):
+    """nvfp4_gemm with the output also NVFP4-quantised (static tensor scale g_y, 16-wide rotation
+    when hadamard=16) for the next layer.  Returns (y or None, y_codes [M, N/2], y_scales)."""
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    dev = a_codes.device
+    y = _gemm_out(M, N, out, dev) if write_y else None
+    if y_codes is None:
+        y_codes = torch.empty(M, N // 2, dtype=torch.uint8, device=dev)
+    if y_scales is None:
+        y_scales = torch.empty(scale_bytes(M, N // 16), dtype=torch.uint8, device=dev)
+    ws, wsb = _gemm_ws(M, N, K, workspace, dev)
+    _check("nvfp4_gemm_quant", lib().nvfp4_gemm_quant(
+        _ptr(a_codes), _ptr(a_scales), _ptr(g_a), _ptr(w_codes), _ptr(w_scales), _ptr(g_w), _ptr(y),
+        y.stride(0) if y is not None else N, hadamard, _ptr(g_y), _ptr(y_codes), _ptr(y_scales), M, N, K, _ptr(ws),
+        wsb, _stream(stream)))
+    return y, y_codes, y_scales
 
 
 def mxfp4_gemm(a_codes, a_scales, w_codes, w_scales, *, out=None, workspace=None, stream=None):

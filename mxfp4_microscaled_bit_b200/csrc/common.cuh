@@ -119,6 +119,18 @@ __device__ __forceinline__ float e4m3_value(uint32_t b)
     return (b & 0x80u) ? -mag : mag;
 }
 
+// NVFP4 block scale from the block maximum and the FP32 tensor scale g:
+// t = (amax/6)/g, sf = E4M3(t), d = dec(sf)*g; returns sf and sets rcp = 1/d
+// (0 when d = 0).  The one arithmetic every NVFP4 encoder in this library uses.
+__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float g, float &rcp)
+{
+    const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
+    const uint32_t sf = cvt_e4m3(t);
+    const float d = __fmul_rn(e4m3_value(sf), g);
+    rcp = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+    return sf;
+}
+
 // ------------------------------------------------------------------ misc
 __device__ __forceinline__ unsigned long long globaltimer_ns()
 {

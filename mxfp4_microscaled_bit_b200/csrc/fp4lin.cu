@@ -197,7 +197,7 @@ template <class C>
 int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const uint8_t *a_codes,
                     const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes, const uint8_t *w_scales,
                     const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy, float *ws,
-                    cudaStream_t st)
+                    cudaStream_t st, const QuantOut &qo)
 {
     {
         std::lock_guard<std::mutex> lk(g_mutex);
@@ -231,6 +231,11 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
     p.splits = pl.splits;
     p.work = (int64_t)pl.num_mt * pl.num_nt * pl.splits;
     p.raster = raster_group(pl.num_mt);
+    p.qc = qo.qc;
+    p.qs = qo.qs;
+    p.qg = qo.qg;
+    p.qhad = qo.qhad;
+    p.qkatoms = qo.qkatoms;
     const int grid = (int)std::min<int64_t>(p.work, dev->sms);
     fp4_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, p);
     if (launch_status() != FP4LIN_OK)
@@ -241,7 +246,7 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
         const int rgrid = (int)std::min<int64_t>((items + 255) / 256, (int64_t)dev->sms * 8);
         splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(ws, pl.splits, rM, rN, pl.ldw, C::NV ? g_a : nullptr,
                                                     C::NV ? g_w : nullptr, reinterpret_cast<__nv_bfloat16 *>(y),
-                                                    ldy);
+                                                    ldy, qo);
         if (launch_status() != FP4LIN_OK)
             return FP4LIN_ERR_CUDA;
     }
@@ -308,17 +313,22 @@ int launch_gemm_pair(DeviceInfo *dev, int slot, const uint8_t *a_codes, const ui
 
 int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
                const uint8_t *w_scales, const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
-               void *workspace, size_t workspace_bytes, void *stream)
+               void *workspace, size_t workspace_bytes, void *stream, const QuantOut &qo = QuantOut{})
 {
-    if (!a_codes || !a_scales || !w_codes || !w_scales || !y || (nv && (!g_a || !g_w)))
+    const bool quant = qo.qc != nullptr;
+    if (!a_codes || !a_scales || !w_codes || !w_scales || (!y && !quant) || (nv && (!g_a || !g_w)))
         return FP4LIN_ERR_INVALID_ARGUMENT;
-    if (M < 1 || N < 1 || K < 1 || ldy < N)
+    if (quant && (!qo.qs || !qo.qg || (qo.qhad != 0 && qo.qhad != 16)))
         return FP4LIN_ERR_INVALID_ARGUMENT;
-    if (K % 64 != 0 || ldy % 8 != 0 || M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+    if (M < 1 || N < 1 || K < 1 || (y && ldy < N))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (K % 64 != 0 || (y && ldy % 8 != 0) || (quant && N % 64 != 0) || M > INT32_MAX / 2 || N > INT32_MAX / 2 ||
+        K > INT32_MAX / 2)
         return FP4LIN_ERR_UNSUPPORTED_SHAPE;
     if (!aligned(a_codes, 16) || !aligned(w_codes, 16) || !aligned(a_scales, 16) || !aligned(w_scales, 16) ||
         !aligned(y, 16) || (nv && (!aligned(g_a, 4) || !aligned(g_w, 4))) ||
-        (workspace && !aligned(workspace, 16)))
+        (workspace && !aligned(workspace, 16)) ||
+        (quant && (!aligned(qo.qc, 16) || !aligned(qo.qs, 16) || !aligned(qo.qg, 4))))
         return FP4LIN_ERR_MISALIGNED;
     DeviceInfo *dev = nullptr;
     int st = current_device(&dev);
@@ -334,11 +344,11 @@ int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const f
     if (pl.swap) {  // the weights take the MMA's M side: operands and shapes swap places
         if (nv)
             return launch_gemm_cfg<GemmCfg<16, true, true>>(dev, 4, pl, w_codes, w_scales, g_w, a_codes, a_scales,
-                                                            g_a, y, N, M, K, ldy, ws, s);
+                                                            g_a, y, N, M, K, ldy, ws, s, qo);
         return launch_gemm_cfg<GemmCfg<16, false, true>>(dev, 5, pl, w_codes, w_scales, nullptr, a_codes, a_scales,
-                                                         nullptr, y, N, M, K, ldy, ws, s);
+                                                         nullptr, y, N, M, K, ldy, ws, s, qo);
     }
-    if (use_pair_kernel(pl)) {
+    if (!quant && use_pair_kernel(pl)) {
         if (nv)
             return launch_gemm_pair<Gemm2Cfg<true>>(dev, 0, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N,
                                                     K, ldy, s);
@@ -348,15 +358,15 @@ int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const f
     if (nv) {
         if (pl.bn == 256)
             return launch_gemm_cfg<GemmCfg<256, true>>(dev, 0, pl, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y,
-                                                       M, N, K, ldy, ws, s);
+                                                       M, N, K, ldy, ws, s, qo);
         return launch_gemm_cfg<GemmCfg<64, true>>(dev, 1, pl, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M,
-                                                  N, K, ldy, ws, s);
+                                                  N, K, ldy, ws, s, qo);
     }
     if (pl.bn == 256)
         return launch_gemm_cfg<GemmCfg<256, false>>(dev, 2, pl, a_codes, a_scales, nullptr, w_codes, w_scales,
-                                                     nullptr, y, M, N, K, ldy, ws, s);
+                                                     nullptr, y, M, N, K, ldy, ws, s, qo);
     return launch_gemm_cfg<GemmCfg<64, false>>(dev, 3, pl, a_codes, a_scales, nullptr, w_codes, w_scales, nullptr, y,
-                                                M, N, K, ldy, ws, s);
+                                                M, N, K, ldy, ws, s, qo);
 }
 
 // ------------------------------------------------------------------ quantiser helpers
@@ -591,6 +601,31 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a
 {
     return gemm_entry(true, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N, K, ldy, workspace,
                       workspace_bytes, stream);
+}
+
+int nvfp4_gemm_quant(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
+                     const uint8_t *w_scales, const float *g_w, void *y, int64_t ldy, int hadamard,
+                     const float *g_y, uint8_t *y_codes, uint8_t *y_scales, int64_t M, int64_t N, int64_t K,
+                     void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!y_codes)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    QuantOut qo{};
+    qo.qc = y_codes;
+    qo.qs = y_scales;
+    qo.qg = g_y;
+    qo.qhad = hadamard;
+    qo.qkatoms = N / 64;
+    int st = gemm_entry(true, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N, K, y ? ldy : N, workspace,
+                        workspace_bytes, stream, qo);
+    if (st != FP4LIN_OK)
+        return st;
+    DeviceInfo *dev = nullptr;
+    if ((st = current_device(&dev)) != FP4LIN_OK)
+        return st;
+    // rows M .. the next multiple of 128 of the output's scale layout are padding: zero them
+    QuantShape q = make_shape(nullptr, M, N, N, y_codes, y_scales, 16);
+    return launch_padding(q, dev, as_stream(stream));
 }
 
 int mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const uint8_t *w_codes, const uint8_t *w_scales,

@@ -25,6 +25,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "quantize.cuh"  // fwht, abs_max, tc_offset: the output quantisation encodes as the quantiser does
 
 namespace fp4lin {
 
@@ -264,7 +265,66 @@ struct GemmParams {
     int64_t katoms;             // scale atoms per 128-row tile along K
     int num_mt, num_nt, nk, kps, splits;
     int64_t work;               // num_mt * num_nt * splits
+    // Optional NVFP4 quantisation of the bf16 output for the next layer (qc null: off):
+    // codes [M, N/2], scales tensor-core layout of [M, N/16] (qkatoms = N/64 atoms per
+    // row tile), static tensor scale *qg, 16-wide rotation when qhad.  y may then be null.
+    uint8_t *qc, *qs;
+    const float *qg;
+    int qhad;
+    int64_t qkatoms;
 };
+
+// NVFP4-encode 16 consecutive output values of one row held by this thread (already
+// rounded to bf16): rotation, block scale, codes -- the quantiser's arithmetic.
+__device__ __forceinline__ void quantize_out_block(const float *y16, int64_t m, int64_t nb, uint8_t *qc,
+                                                   uint8_t *qs, float g, bool had, int64_t N, int64_t katoms)
+{
+    float w[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        w[j] = y16[j];
+    if (had) {
+        fwht<16>(w);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            w[j] = __fmul_rn(w[j], 0.25f);
+    }
+    float rcp;
+    const uint32_t sf = nvfp4_block_scale(abs_max<16>(w), g, rcp);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        w[j] = __fmul_rn(w[j], rcp);
+    *reinterpret_cast<uint2 *>(qc + m * (N / 2) + nb / 2) = make_uint2(pack_e2m1x8(w), pack_e2m1x8(w + 8));
+    qs[tc_offset(m, nb / 16, katoms)] = (uint8_t)sf;
+}
+
+// The 16-point rotation of a block spread over L lanes (16/L consecutive values per lane,
+// lanes of a block consecutive): butterfly strides 1, 2, ... in order, the pair (u, w)
+// becoming (u + w, u - w); strides >= 16/L pair values of lanes lane ^ (stride / (16/L)).
+template <int L>
+__device__ __forceinline__ void fwht16_lanes(float *w)
+{
+    constexpr int E = 16 / L;  // values per lane
+#pragma unroll
+    for (int h = 1; h < E; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < E; ++i)
+            if ((i & h) == 0) {
+                const float u = w[i], x = w[i + h];
+                w[i] = __fadd_rn(u, x);
+                w[i + h] = __fsub_rn(u, x);
+            }
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int h = 1; h < L; h <<= 1) {
+        const bool upper = (lane & h) != 0;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const float o = __shfl_xor_sync(0xffffffffu, w[i], h);
+            w[i] = upper ? __fsub_rn(o, w[i]) : __fadd_rn(w[i], o);  // upper: (lower u) - (own w)
+        }
+    }
+}
 
 // MMAs (64 values of K each) in k-tile kt: 4, or fewer in a last partial tile.
 template <class C>
@@ -478,6 +538,40 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if constexpr (C::SWAP) {
                 // accumulator row = weight row n, column = activation row m: y[m, n]
                 const int64_t n = (int64_t)mt * C::BM + quad * 32 + lane;
+                if (p.splits == 1 && p.qc) {
+                    // output quantisation: a 16-column block of row m lies on 16 lanes; with
+                    // N % 64 == 0 the warp's 32 columns are all inside or all outside N
+                    if ((int64_t)mt * C::BM + quad * 32 < p.M) {
+                        const float qg = *p.qg;
+#pragma unroll
+                        for (int c = 0; c < C::COLS_PER_WARP; ++c) {
+                            const int64_t m = (int64_t)nt * C::BN + half * C::COLS_PER_WARP + c;
+                            if (m >= p.N)
+                                break;
+                            const __nv_bfloat16 yb = __float2bfloat16_rn(__fmul_rn(v[c], gg));
+                            if (p.y)
+                                p.y[m * p.ldy + n] = yb;
+                            float w = __bfloat162float(yb);
+                            if (p.qhad) {
+                                fwht16_lanes<16>(&w);
+                                w = __fmul_rn(w, 0.25f);
+                            }
+                            float a = fabsf(w);
+#pragma unroll
+                            for (int o = 1; o < 16; o <<= 1)
+                                a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+                            float rcp;
+                            const uint32_t sf = nvfp4_block_scale(a, qg, rcp);
+                            const float wv = __fmul_rn(w, rcp);
+                            const float wn = __shfl_xor_sync(0xffffffffu, wv, 1);
+                            if ((lane & 1) == 0)  // even column: low nibble, its odd neighbour: high
+                                p.qc[m * (p.M / 2) + n / 2] = (uint8_t)cvt_e2m1x2(wv, wn);
+                            if ((lane & 15) == 0)
+                                p.qs[tc_offset(m, n / 16, p.qkatoms)] = (uint8_t)sf;
+                        }
+                    }
+                    continue;
+                }
                 if (n < p.M) {
 #pragma unroll
                     for (int c = 0; c < C::COLS_PER_WARP; ++c) {
@@ -497,24 +591,36 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int64_t n0 = (int64_t)nt * C::BN + half * C::COLS_PER_WARP;
             if (m < p.M) {
                 if (p.splits == 1) {
-                    __nv_bfloat16 *yr = p.y + m * p.ldy;
+                    // round once to bf16, in place: the stored y and the quantised y agree
 #pragma unroll
-                    for (int c = 0; c < C::COLS_PER_WARP; c += 8) {
-                        const int64_t n = n0 + c;
-                        if (n + 8 <= p.N) {
-                            uint32_t w4[4];
+                    for (int c = 0; c < C::COLS_PER_WARP; ++c)
+                        v[c] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(v[c], gg)));
+                    if (p.y) {
+                        __nv_bfloat16 *yr = p.y + m * p.ldy;
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(v[c + 2 * j], gg),
-                                                                          __fmul_rn(v[c + 2 * j + 1], gg));
-                                w4[j] = *reinterpret_cast<uint32_t *>(&b2);
+                        for (int c = 0; c < C::COLS_PER_WARP; c += 8) {
+                            const int64_t n = n0 + c;
+                            if (n + 8 <= p.N) {
+                                uint32_t w4[4];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    __nv_bfloat162 b2 = __floats2bfloat162_rn(v[c + 2 * j], v[c + 2 * j + 1]);
+                                    w4[j] = *reinterpret_cast<uint32_t *>(&b2);
+                                }
+                                st_v4(yr + n, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+                            } else {
+                                for (int j = 0; j < 8; ++j)
+                                    if (n + j < p.N)
+                                        yr[n + j] = __float2bfloat16_rn(v[c + j]);
                             }
-                            st_v4(yr + n, make_uint4(w4[0], w4[1], w4[2], w4[3]));
-                        } else {
-                            for (int j = 0; j < 8; ++j)
-                                if (n + j < p.N)
-                                    yr[n + j] = __float2bfloat16_rn(__fmul_rn(v[c + j], gg));
                         }
+                    }
+                    if (p.qc) {
+                        const float qg = *p.qg;
+#pragma unroll
+                        for (int c = 0; c < C::COLS_PER_WARP; c += 16)
+                            if (n0 + c < p.N)  // N % 64 == 0: whole blocks
+                                quantize_out_block(v + c, m, n0 + c, p.qc, p.qs, qg, p.qhad != 0, p.N, p.qkatoms);
                     }
                 } else {
                     float *wr = p.ws + ((int64_t)sp * p.M + m) * p.ldw;
@@ -545,38 +651,90 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
 }
 
-// y = bf16(g_a * g_w * sum_s ws[s]) in split order (deterministic).
+// Output quantisation arguments of the split-K reduction (qc null: off); see GemmParams.
+struct QuantOut {
+    uint8_t *qc, *qs;
+    const float *qg;
+    int qhad;
+    int64_t qkatoms;
+};
+
+// y = bf16(g_a * g_w * sum_s ws[s]) in split order (deterministic), and optionally its NVFP4
+// encoding.  Every lane of a warp runs the same iterations: with N % 64 == 0 a 16-column
+// block of the output is 4 consecutive lanes, which share its maximum and rotation by shuffles.
 __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *ws, int splits, int64_t M, int64_t N,
                                                             int64_t ldw, const float *g_a, const float *g_w,
-                                                            __nv_bfloat16 *y, int64_t ldy)
+                                                            __nv_bfloat16 *y, int64_t ldy, QuantOut qo)
 {
     const float gg = (g_a && g_w) ? __fmul_rn(*g_a, *g_w) : 1.0f;
+    const float qg = qo.qc ? *qo.qg : 1.0f;
     const int64_t nq = (N + 3) / 4, total = M * nq;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = i / nq, n = (i - m * nq) * 4;
+    const int lane = threadIdx.x & 31;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < total; base += stride) {
+        const int64_t i = base + lane;
+        const bool valid = i < total;
+        int64_t m = 0, n = 0;
         float s[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int k = 0; k < splits; ++k) {
-            const float *src = ws + ((int64_t)k * M + m) * ldw + n;
-            if (n + 4 <= N) {
-                const float4 f = *reinterpret_cast<const float4 *>(src);
-                s[0] = __fadd_rn(s[0], f.x);
-                s[1] = __fadd_rn(s[1], f.y);
-                s[2] = __fadd_rn(s[2], f.z);
-                s[3] = __fadd_rn(s[3], f.w);
-            } else {
-                for (int j = 0; j < 4 && n + j < N; ++j)
-                    s[j] = __fadd_rn(s[j], src[j]);
+        if (valid) {
+            m = i / nq;
+            n = (i - m * nq) * 4;
+            for (int k = 0; k < splits; ++k) {
+                const float *src = ws + ((int64_t)k * M + m) * ldw + n;
+                if (n + 4 <= N) {
+                    const float4 f = *reinterpret_cast<const float4 *>(src);
+                    s[0] = __fadd_rn(s[0], f.x);
+                    s[1] = __fadd_rn(s[1], f.y);
+                    s[2] = __fadd_rn(s[2], f.z);
+                    s[3] = __fadd_rn(s[3], f.w);
+                } else {
+                    for (int j = 0; j < 4 && n + j < N; ++j)
+                        s[j] = __fadd_rn(s[j], src[j]);
+                }
             }
         }
-        __nv_bfloat16 *dst = y + m * ldy + n;
-        if (n + 4 <= N) {
-            __nv_bfloat162 lo = __floats2bfloat162_rn(__fmul_rn(s[0], gg), __fmul_rn(s[1], gg));
-            __nv_bfloat162 hi = __floats2bfloat162_rn(__fmul_rn(s[2], gg), __fmul_rn(s[3], gg));
-            uint2 u = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
-            *reinterpret_cast<uint2 *>(dst) = u;
-        } else {
-            for (int j = 0; j < 4 && n + j < N; ++j)
-                dst[j] = __float2bfloat16_rn(__fmul_rn(s[j], gg));
+        if (!qo.qc) {
+            if (!valid)
+                continue;
+            __nv_bfloat16 *dst = y + m * ldy + n;
+            if (n + 4 <= N) {
+                __nv_bfloat162 lo = __floats2bfloat162_rn(__fmul_rn(s[0], gg), __fmul_rn(s[1], gg));
+                __nv_bfloat162 hi = __floats2bfloat162_rn(__fmul_rn(s[2], gg), __fmul_rn(s[3], gg));
+                uint2 u = make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+                *reinterpret_cast<uint2 *>(dst) = u;
+            } else {
+                for (int j = 0; j < 4 && n + j < N; ++j)
+                    dst[j] = __float2bfloat16_rn(__fmul_rn(s[j], gg));
+            }
+            continue;
+        }
+        // output quantisation (N % 64 == 0: four whole columns per lane)
+        float w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            w[j] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(s[j], gg)));
+        if (valid && y) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(w[0], w[1]), hi = __floats2bfloat162_rn(w[2], w[3]);
+            *reinterpret_cast<uint2 *>(y + m * ldy + n) =
+                make_uint2(*reinterpret_cast<uint32_t *>(&lo), *reinterpret_cast<uint32_t *>(&hi));
+        }
+        if (qo.qhad) {
+            fwht16_lanes<4>(w);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                w[j] = __fmul_rn(w[j], 0.25f);
+        }
+        float a = abs_max<4>(w);
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+        float rcp;
+        const uint32_t sf = nvfp4_block_scale(a, qg, rcp);
+        if (valid) {
+            const uint32_t c01 = cvt_e2m1x2(__fmul_rn(w[0], rcp), __fmul_rn(w[1], rcp));
+            const uint32_t c23 = cvt_e2m1x2(__fmul_rn(w[2], rcp), __fmul_rn(w[3], rcp));
+            *reinterpret_cast<uint16_t *>(qo.qc + m * (N / 2) + n / 2) = (uint16_t)(c01 | (c23 << 8));
+            if ((lane & 3) == 0)
+                qo.qs[tc_offset(m, n / 16, qo.qkatoms)] = (uint8_t)sf;
         }
     }
 }

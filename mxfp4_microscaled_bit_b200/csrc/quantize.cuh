@@ -234,11 +234,8 @@ __global__ void __launch_bounds__(QTHREADS)
             continue;
         float v[16];
         nvfp4_block_values<HAD>(raw[u], v);
-        const float amax = abs_max<16>(v);
-        const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
-        const uint32_t sf = cvt_e4m3(t);
-        const float d = __fmul_rn(e4m3_value(sf), g);
-        const float rcp = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+        float rcp;
+        const uint32_t sf = nvfp4_block_scale(abs_max<16>(v), g, rcp);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
             v[j] = __fmul_rn(v[j], rcp);
