@@ -240,6 +240,26 @@ class Workload:
         fl.mxfp4_gemm(self.a_codes, self.a_scales_mx, self.w_mx.codes, self.w_mx.scales, out=self.y,
                       workspace=False)
 
+    # the layer's output as the next layer's NVFP4 input (static tensor scale, 16-wide rotation)
+    def chained_setup(self):
+        fl = self.fl
+        self.step()
+        _, _, self.g_y = fl.nvfp4_quantize(self.y, 16)  # computed once, as a calibrated static scale
+        self.y_codes = torch.empty(self.M, self.N // 2, dtype=torch.uint8, device=self.dev)
+        self.y_scales = torch.empty(fl.scale_bytes(self.M, self.N // 16), dtype=torch.uint8, device=self.dev)
+
+    def gemm_then_quantize(self):
+        fl = self.fl
+        fl.nvfp4_gemm(self.a_codes, self.a_scales, self.g_a, self.w.codes, self.w.scales, self.w.g, out=self.y,
+                      workspace=False)
+        fl.nvfp4_quantize(self.y, 16, self.g_y, compute_global_scale=False, codes=self.y_codes,
+                          scales=self.y_scales)
+
+    def gemm_quant_fused(self):
+        self.fl.nvfp4_gemm_quant(self.a_codes, self.a_scales, self.g_a, self.w.codes, self.w.scales, self.w.g,
+                                 self.g_y, hadamard=16, write_y=False, y_codes=self.y_codes,
+                                 y_scales=self.y_scales, workspace=False)
+
     # algorithmic work
     def flops(self):
         return 2.0 * self.M * self.N * self.K
@@ -406,6 +426,15 @@ def main():
         w.mxfp4_layer()
     mx_ms = time_loop(w.mxfp4_layer, 20, stream) / 20
 
+    # ---- the output handed to a next NVFP4 layer: GEMM then quantiser vs the fused epilogue
+    w.chained_setup()
+    for _ in range(3):
+        w.gemm_then_quantize()
+        w.gemm_quant_fused()
+    unfused_ms = time_loop(w.gemm_then_quantize, 20, stream) / 20
+    fused_ms = time_loop(w.gemm_quant_fused, 20, stream) / 20
+    assert fl.device_status() == 0
+
     # ---- end to end through the public API with host buffers: H2D of A and the new K/V rows,
     #      the step, D2H of y and the FP8 output scales
     def e2e_step():
@@ -487,7 +516,12 @@ def main():
                     "quantize_gbs": rooflines["quantize"]["achieved"],
                     "kv_load_gbs": rooflines["kv_load_fp8"]["achieved"],
                     "kv_store_us": st_ms * 1e3,
-                    "mxfp4_layer_tflops": flops / (mx_ms * 1e-3) / 1e12},
+                    "mxfp4_layer_tflops": flops / (mx_ms * 1e-3) / 1e12,
+                    "next_layer_input": {
+                        "gemm_then_quantize_ms": unfused_ms, "gemm_quant_fused_ms": fused_ms,
+                        "speedup": unfused_ms / fused_ms,
+                        "note": "y handed on as NVFP4 (static g_y, H16): nvfp4_gemm + nvfp4_quantize vs "
+                                "nvfp4_gemm_quant without bf16 y; back-to-back calls, operands L2-warm"}},
         "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": Workload.LAUNCHES_PER_STEP * args.steps,
