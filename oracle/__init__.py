@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
                 "oracle_kv_store": (None, [u16p, i32p, ctypes.c_float, u8p, u8p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, i64, ctypes.c_int]),
                 "oracle_kv_load_fp8": (None, [u8p, u8p, i64, ctypes.c_int, ctypes.c_int, i64, ctypes.c_int, u8p]),
+                "oracle_kv_attention": (None, [u16p, u8p, u8p, ctypes.c_float, u8p, u8p, ctypes.c_float, i64,
+                                               ctypes.c_int, ctypes.c_int, ctypes.c_int, i64, ctypes.c_int, f64p]),
             }
             for name, (res, args) in sig.items():
                 fn = getattr(L, name)
@@ -265,4 +267,20 @@ def kv_load_fp8(cache_codes: np.ndarray, cache_sf: np.ndarray, L: int) -> np.nda
     out = np.empty((B, H, L, D), dtype=np.uint8)
     lib().oracle_kv_load_fp8(_p(c, ctypes.c_uint8), _p(s, ctypes.c_uint8), L, B, H, Lcap, D,
                              _p(out, ctypes.c_uint8))
+    return out
+
+
+def kv_attention(q, k_codes, k_sf, gk: float, v_codes, v_sf, gv: float, L: int) -> np.ndarray:
+    """Decode attention (reading R11) over the first L cached positions.  q: bf16 [B, H*G, D];
+    caches as kv_store.  -> float64 [B, H*G, D]."""
+    qb = _bits(q)
+    B, HG, D = qb.shape
+    kc, ks = np.ascontiguousarray(k_codes, dtype=np.uint8), np.ascontiguousarray(k_sf, dtype=np.uint8)
+    vc, vs = np.ascontiguousarray(v_codes, dtype=np.uint8), np.ascontiguousarray(v_sf, dtype=np.uint8)
+    H, Lcap = kc.shape[1], kc.shape[2]
+    G = HG // H
+    out = np.empty((B, HG, D), dtype=np.float64)
+    lib().oracle_kv_attention(_p(qb, ctypes.c_uint16), _p(kc, ctypes.c_uint8), _p(ks, ctypes.c_uint8), float(gk),
+                              _p(vc, ctypes.c_uint8), _p(vs, ctypes.c_uint8), float(gv), L, B, H, G, Lcap, D,
+                              _p(out, ctypes.c_double))
     return out

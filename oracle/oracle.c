@@ -50,6 +50,10 @@
  *      nearest power of two): the ideal scale amax/6 is rounded to the nearer
  *      of the two powers of two around it, by value, ties upward.  With
  *      e = floor(log2 amax) that is X = e-2 when amax >= 1.125*2^e, else e-3.
+ *   R11 Decode attention over the NVFP4 KV cache ([KV] says only that the FP8
+ *      copy feeds attention): G query heads per kv head (query head j uses kv
+ *      head j / G), scores q . k / sqrt(D) over positions 0..L-1, softmax, the
+ *      p-weighted sum of the values; q bf16, output fp32; no mask beyond L.
  */
 #include <math.h>
 #include <stdint.h>
@@ -484,4 +488,67 @@ EXPORT void oracle_kv_load_fp8(const uint8_t *cache_codes, const uint8_t *cache_
                 out[(bh * L + l) * D + d] = oracle_e4m3_encode((float)v);
             }
         }
+}
+
+/* The FP8 value (R8) of one cached element, times 8g: the value attention reads. */
+static double kv_fp8_value(const uint8_t *codes_row, const uint8_t *sf_row, int d, double g8)
+{
+    uint8_t byte = codes_row[d / 2];
+    uint8_t c = (d & 1) ? (byte >> 4) : (byte & 15);
+    double v = oracle_e2m1_decode(c) * oracle_e4m3_decode(sf_row[d / 16]) * 0.125;
+    return oracle_e4m3_decode(oracle_e4m3_encode((float)v)) * g8;
+}
+
+/* Decode attention over the cache as attention reads it after the FP8 load ([KV]:
+ * new K/V rows stored in NVFP4 and dequantised to FP8 before attention; reading
+ * R11 for the attention itself): query head j of batch b uses kv head h = j / G;
+ * k_l, v_l are the FP8 values of position l times 8g; s_l = (q . k_l) / sqrt(D);
+ * p = softmax(s) over l < L; o = sum_l p_l v_l.  binary64 throughout.
+ * q: bf16 [B, H*G, D]; caches as oracle_kv_store; out: [B, H*G, D]. */
+EXPORT void oracle_kv_attention(const uint16_t *q, const uint8_t *kc, const uint8_t *ks, float gk,
+                                const uint8_t *vc, const uint8_t *vs, float gv, int64_t L, int B, int H,
+                                int G, int64_t Lcap, int D, double *out)
+{
+    const double gk8 = 8.0 * (double)gk, gv8 = 8.0 * (double)gv, inv_sqrt_d = 1.0 / sqrt((double)D);
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+        double *kv = (double *)malloc((size_t)L * D * sizeof(double));
+        double *vv = (double *)malloc((size_t)L * D * sizeof(double));
+        double *s = (double *)malloc((size_t)L * sizeof(double));
+        for (int64_t l = 0; l < L; ++l) {
+            int64_t row = bh * Lcap + l;
+            for (int d = 0; d < D; ++d) {
+                kv[l * D + d] = kv_fp8_value(kc + row * (D / 2), ks + row * (D / 16), d, gk8);
+                vv[l * D + d] = kv_fp8_value(vc + row * (D / 2), vs + row * (D / 16), d, gv8);
+            }
+        }
+        const int64_t b = bh / H, h = bh % H;
+        for (int j = 0; j < G; ++j) {
+            const uint16_t *qr = q + ((b * H + h) * G + j) * (int64_t)D;
+            double m = -INFINITY;
+            for (int64_t l = 0; l < L; ++l) {
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d)
+                    acc += (double)bf16_to_f32(qr[d]) * kv[l * D + d];
+                s[l] = acc * inv_sqrt_d;
+                if (s[l] > m)
+                    m = s[l];
+            }
+            double sum = 0.0;
+            for (int64_t l = 0; l < L; ++l) {
+                s[l] = exp(s[l] - m);
+                sum += s[l];
+            }
+            double *o = out + ((b * H + h) * G + j) * (int64_t)D;
+            for (int d = 0; d < D; ++d) {
+                double acc = 0.0;
+                for (int64_t l = 0; l < L; ++l)
+                    acc += s[l] * vv[l * D + d];
+                o[d] = acc / sum;
+            }
+        }
+        free(kv);
+        free(vv);
+        free(s);
+    }
 }
