@@ -209,6 +209,26 @@ int nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld
                            void *stream);
 
 /*
+ * Decode attention read straight from the NVFP4 KV cache (the story on NVFP4 KV
+ * caches: new K/V rows are stored in NVFP4 and dequantised to FP8 before
+ * attention).  The K and V values are exactly the FP8 values kv_nvfp4_load_fp8
+ * would write, times 8 g_k / 8 g_v, but they are formed on chip: the FP8 copy
+ * is neither written nor read.  Query head j of batch b uses kv head j / G:
+ *   s_l = (q . k_l) / sqrt(D) for l < L, p = softmax(s), out = sum_l p_l v_l,
+ * in binary32 (a split over L merged with rescaled sums).
+ *   q: bf16 [B, H*G, D]; caches as kv_nvfp4_store; g_k, g_v device floats;
+ *   out: float32 [B, H*G, D].
+ * Shapes: D = 128, 1 <= G <= 8, 1 <= L <= Lcap, B*H <= 65535.  codes, q, out,
+ * workspace 16-byte aligned, scales 8-byte aligned.  workspace of at least
+ * kv_attention_workspace_bytes(B, H, G, L, D) bytes (else FP4LIN_ERR_WORKSPACE).
+ */
+size_t kv_attention_workspace_bytes(int B, int H, int G, int64_t L, int D);
+int kv_nvfp4_attention(const void *q, const uint8_t *k_codes, const uint8_t *k_scales,
+                       const float *g_k, const uint8_t *v_codes, const uint8_t *v_scales,
+                       const float *g_v, int64_t L, float *out, int B, int H, int G,
+                       int64_t Lcap, int D, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * nvfp4_gemm whose output is also NVFP4-quantised for the next layer, inside the
  * GEMM's epilogue (or its split-K reduction), so a chain of layers need not
  * write and re-read bf16.  The output is first rounded to bf16 exactly as

@@ -50,6 +50,9 @@ EXPORTS = {
     "nvfp4_quantize_noalloc": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_quantize_nearest": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp]),
+    "kv_attention_workspace_bytes": (_sz, [_int, _int, _int, _i64, _int]),
+    "kv_nvfp4_attention": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _int, _int, _int, _i64, _int, _vp,
+                                  _sz, _vp]),
     "nvfp4_gemm_quant": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _vp, _vp, _vp, _i64, _i64, _i64,
                                 _vp, _sz, _vp]),
 }
@@ -192,6 +195,27 @@ def nvfp4_gemm(a_codes, a_scales, g_a, w_codes, w_scales, g_w, *, out=None, work
     _check("nvfp4_gemm", lib().nvfp4_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(g_a), _ptr(w_codes), _ptr(w_scales),
                                           _ptr(g_w), _ptr(y), M, N, K, y.stride(0), _ptr(ws), wsb, _stream(stream)))
     return y
+
+
+def kv_nvfp4_attention(q, k_cache, v_cache, L: int, *, out=None, workspace=None, stream=None):
+    """Decode attention from the NVFP4 caches.  q: bf16 [B, H*G, D]; k_cache, v_cache: (codes
+    [B,H,Lcap,D/2], scales [B,H,Lcap,D/16], g) as kv_nvfp4_store fills them.
+    Returns float32 [B, H*G, D]."""
+    kc, ks, gk = k_cache
+    vc, vs, gv = v_cache
+    B, H, Lcap, D2 = kc.shape
+    D = 2 * D2
+    G = q.shape[1] // H
+    dev = q.device
+    if out is None:
+        out = torch.empty(B, H * G, D, dtype=torch.float32, device=dev)
+    if workspace is None:
+        need = int(lib().kv_attention_workspace_bytes(B, H, G, L, D))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check("kv_nvfp4_attention", lib().kv_nvfp4_attention(
+        _ptr(q), _ptr(kc), _ptr(ks), _ptr(gk), _ptr(vc), _ptr(vs), _ptr(gv), L, _ptr(out), B, H, G, Lcap, D,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
 
 
 def nvfp4_gemm_quant(a_codes, a_scales, g_a, w_codes, w_scales, g_w, g_y, *, hadamard: int = 0,

@@ -14,6 +14,7 @@
 #include "gemm_sm100.cuh"
 #include "gemm_sm100_2sm.cuh"
 #include "kv.cuh"
+#include "kv_attention.cuh"
 #include "quantize.cuh"
 #include "scale_search.cuh"
 
@@ -601,6 +602,68 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a
 {
     return gemm_entry(true, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N, K, ldy, workspace,
                       workspace_bytes, stream);
+}
+
+size_t kv_attention_workspace_bytes(int B, int H, int G, int64_t L, int D)
+{
+    if (B < 1 || H < 1 || G < 1 || L < 1 || D < 1)
+        return 0;
+    const int64_t S = (L + KA_CHUNK - 1) / KA_CHUNK;
+    return (size_t)B * H * S * G * (D + 2) * sizeof(float);
+}
+
+int kv_nvfp4_attention(const void *q, const uint8_t *k_codes, const uint8_t *k_scales, const float *g_k,
+                       const uint8_t *v_codes, const uint8_t *v_scales, const float *g_v, int64_t L, float *out,
+                       int B, int H, int G, int64_t Lcap, int D, void *workspace, size_t workspace_bytes,
+                       void *stream)
+{
+    if (!q || !k_codes || !k_scales || !g_k || !v_codes || !v_scales || !g_v || !out)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (B < 1 || H < 1 || G < 1 || L < 1 || Lcap < L || D < 1)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (D != KA_D || G > KA_GMAX || (int64_t)B * H > 65535)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(q, 16) || !aligned(k_codes, 16) || !aligned(v_codes, 16) || !aligned(k_scales, 8) ||
+        !aligned(v_scales, 8) || !aligned(g_k, 4) || !aligned(g_v, 4) || !aligned(out, 16) ||
+        (workspace && !aligned(workspace, 16)))
+        return FP4LIN_ERR_MISALIGNED;
+    const size_t need = kv_attention_workspace_bytes(B, H, G, L, D);
+    if (!workspace || workspace_bytes < need)
+        return FP4LIN_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    KvAttnShape a{};
+    a.q = reinterpret_cast<const __nv_bfloat16 *>(q);
+    a.kc = k_codes;
+    a.ks = k_scales;
+    a.vc = v_codes;
+    a.vs = v_scales;
+    a.gk = g_k;
+    a.gv = g_v;
+    a.ws = reinterpret_cast<float *>(workspace);
+    a.out = out;
+    a.L = L;
+    a.Lcap = Lcap;
+    a.H = H;
+    a.S = (int)((L + KA_CHUNK - 1) / KA_CHUNK);
+    const dim3 grid((unsigned)a.S, (unsigned)(B * H));
+    cudaStream_t s = as_stream(stream);
+    switch (G) {
+    case 1: kv_attn_split_kernel<1><<<grid, KA_THREADS, 0, s>>>(a); break;
+    case 2: kv_attn_split_kernel<2><<<grid, KA_THREADS, 0, s>>>(a); break;
+    case 3: kv_attn_split_kernel<3><<<grid, KA_THREADS, 0, s>>>(a); break;
+    case 4: kv_attn_split_kernel<4><<<grid, KA_THREADS, 0, s>>>(a); break;
+    case 5: kv_attn_split_kernel<5><<<grid, KA_THREADS, 0, s>>>(a); break;
+    case 6: kv_attn_split_kernel<6><<<grid, KA_THREADS, 0, s>>>(a); break;
+    case 7: kv_attn_split_kernel<7><<<grid, KA_THREADS, 0, s>>>(a); break;
+    default: kv_attn_split_kernel<8><<<grid, KA_THREADS, 0, s>>>(a); break;
+    }
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    kv_attn_merge_kernel<<<(unsigned)((int64_t)B * H * G), KA_D, 0, s>>>(a, G);
+    return launch_status();
 }
 
 int nvfp4_gemm_quant(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
