@@ -260,6 +260,22 @@ class Workload:
                                  self.g_y, hadamard=16, write_y=False, y_codes=self.y_codes,
                                  y_scales=self.y_scales, workspace=False)
 
+    def attention_setup(self, G):
+        """-> a callable running kv_nvfp4_attention over the decode step's caches."""
+        fl = self.fl
+        gen = torch.Generator(device=self.dev).manual_seed(5)
+        q = torch.randn(self.B, self.H * G, self.D, generator=gen, device=self.dev).to(torch.bfloat16)
+        out = torch.empty(self.B, self.H * G, self.D, dtype=torch.float32, device=self.dev)
+        ws = torch.empty(fl.lib().kv_attention_workspace_bytes(self.B, self.H, G, self.L, self.D),
+                         dtype=torch.uint8, device=self.dev)
+        k = (self.cache["k"][0], self.cache["k"][1], self.kv_g["k"])
+        v = (self.cache["v"][0], self.cache["v"][1], self.kv_g["v"])
+        self.attn_G = G
+        return lambda: fl.kv_nvfp4_attention(q, k, v, self.L, out=out, workspace=ws)
+
+    def attention_bytes(self):
+        return 2 * self.B * self.H * self.L * self.D * (0.5 + 1 / 16)  # K and V codes + scales, once
+
     # algorithmic work
     def flops(self):
         return 2.0 * self.M * self.N * self.K
@@ -435,6 +451,13 @@ def main():
     fused_ms = time_loop(w.gemm_quant_fused, 20, stream) / 20
     assert fl.device_status() == 0
 
+    # ---- decode attention straight from the NVFP4 caches (G = 4 query heads per kv head)
+    attn = w.attention_setup(4)
+    for _ in range(3):
+        attn()
+    attn_ms = time_loop(attn, 10, stream) / 10
+    assert fl.device_status() == 0
+
     # ---- end to end through the public API with host buffers: H2D of A and the new K/V rows,
     #      the step, D2H of y and the FP8 output scales
     def e2e_step():
@@ -517,6 +540,14 @@ def main():
                     "kv_load_gbs": rooflines["kv_load_fp8"]["achieved"],
                     "kv_store_us": st_ms * 1e3,
                     "mxfp4_layer_tflops": flops / (mx_ms * 1e-3) / 1e12,
+                    "kv_attention": {
+                        "ms": attn_ms, "G": w.attn_G,
+                        "gbs": w.attention_bytes() / (attn_ms * 1e-3) / 1e9,
+                        "frac_hbm": w.attention_bytes() / (attn_ms * 1e-3) / 1e9 / hbm,
+                        "kv_load_fp8_ms": ld_ms,
+                        "note": "decode attention over the NVFP4 caches with the FP8 values formed on chip; "
+                                "kv_load_fp8_ms is the step's FP8 load of the same caches, which an FP8 "
+                                "attention kernel would then read back"},
                     "next_layer_input": {
                         "gemm_then_quantize_ms": unfused_ms, "gemm_quant_fused_ms": fused_ms,
                         "speedup": unfused_ms / fused_ms,
