@@ -63,6 +63,48 @@ __device__ __forceinline__ void fwht(float *v)
             }
 }
 
+// The same butterflies on the packed binary32 pipe: stride 1 pairs neighbours and runs
+// scalar; every stride h >= 2 pairs element 2m with 2m+h and 2m+1 with 2m+1+h, so the
+// pairs (v[2m], v[2m+1]) move together through add/sub.f32x2 -- the same IEEE operations
+// in the same order, two per instruction.  The 1/sqrt(B) scaling `s` is packed too.
+template <int B>
+__device__ __forceinline__ void fwht_scaled_packed(float *v, float s)
+{
+#pragma unroll
+    for (int i = 0; i < B; i += 2) {
+        const float u = v[i], w = v[i + 1];
+        v[i] = __fadd_rn(u, w);
+        v[i + 1] = __fsub_rn(u, w);
+    }
+    uint64_t P[B / 2];
+#pragma unroll
+    for (int m = 0; m < B / 2; ++m)
+        P[m] = f2_pack(v[2 * m], v[2 * m + 1]);
+#pragma unroll
+    for (int h2 = 1; h2 < B / 2; h2 <<= 1)
+#pragma unroll
+        for (int m = 0; m < B / 2; ++m)
+            if ((m & h2) == 0) {
+                const uint64_t a = P[m], b = P[m + h2];
+                P[m] = f2_add(a, b);
+                P[m + h2] = f2_sub(a, b);
+            }
+    const uint64_t ss = f2_pack(s, s);
+#pragma unroll
+    for (int m = 0; m < B / 2; ++m)
+        f2_unpack(f2_mul(P[m], ss), v[2 * m], v[2 * m + 1]);
+}
+
+// v[j] = RN(v[j] * s) for B values, two per packed instruction.
+template <int B>
+__device__ __forceinline__ void scale_packed(float *v, float s)
+{
+    const uint64_t ss = f2_pack(s, s);
+#pragma unroll
+    for (int m = 0; m < B / 2; ++m)
+        f2_unpack(f2_mul(f2_pack(v[2 * m], v[2 * m + 1]), ss), v[2 * m], v[2 * m + 1]);
+}
+
 template <int B>
 __device__ __forceinline__ float abs_max(const float *v)
 {
@@ -79,12 +121,8 @@ __device__ __forceinline__ void nvfp4_block_values(const uint32_t *raw, float *v
 {
     bf16x8_to_f32(make_uint4(raw[0], raw[1], raw[2], raw[3]), v);
     bf16x8_to_f32(make_uint4(raw[4], raw[5], raw[6], raw[7]), v + 8);
-    if (HAD) {
-        fwht<16>(v);
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            v[j] = __fmul_rn(v[j], 0.25f);  // 1/sqrt(16), exact
-    }
+    if (HAD)
+        fwht_scaled_packed<16>(v, 0.25f);  // 1/sqrt(16), exact
 }
 
 // The (rotated, when HAD) values of one MXFP4 block: 32 bf16 in `raw`.
@@ -94,12 +132,8 @@ __device__ __forceinline__ void mxfp4_block_values(const uint32_t *raw, float *v
 #pragma unroll
     for (int k = 0; k < 4; ++k)
         bf16x8_to_f32(make_uint4(raw[4 * k], raw[4 * k + 1], raw[4 * k + 2], raw[4 * k + 3]), v + 8 * k);
-    if (HAD) {
-        fwht<32>(v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-            v[j] = __fmul_rn(v[j], 0x1.6a09e6p-3f);  // 1/sqrt(32) rounded to binary32
-    }
+    if (HAD)
+        fwht_scaled_packed<32>(v, 0x1.6a09e6p-3f);  // 1/sqrt(32) rounded to binary32
 }
 
 // Zero the padding bytes of a tensor-core scale buffer (rows past `rows`,
@@ -236,9 +270,7 @@ __global__ void __launch_bounds__(QTHREADS)
         nvfp4_block_values<HAD>(raw[u], v);
         float rcp;
         const uint32_t sf = nvfp4_block_scale(abs_max<16>(v), g, rcp);
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            v[j] = __fmul_rn(v[j], rcp);
+        scale_packed<16>(v, rcp);
         *reinterpret_cast<uint2 *>(q.codes + r * (q.cols / 2) + c * 8) = make_uint2(pack_e2m1x8(v), pack_e2m1x8(v + 8));
         q.scales[tc_offset(r, c, q.katoms)] = (uint8_t)sf;
     }
@@ -289,9 +321,7 @@ __global__ void __launch_bounds__(QTHREADS) mxfp4_quant_kernel(QuantShape q)
             const uint32_t lower = (NEAREST && (bits & 0x7FFFFFu) < 0x100000u) ? 1u : 0u;
             const uint32_t byte = E >= 2u + lower ? E - 2u - lower : 0u;
             const float s = __uint_as_float((254u - byte) << 23);  // 2^(127 - byte)
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-                v[j] = __fmul_rn(v[j], s);
+            scale_packed<32>(v, s);
             st_v4(q.codes + r * (q.cols / 2) + c * 16,
                   make_uint4(pack_e2m1x8(v), pack_e2m1x8(v + 8), pack_e2m1x8(v + 16), pack_e2m1x8(v + 24)));
             q.scales[tc_offset(r, c, q.katoms)] = (uint8_t)byte;
