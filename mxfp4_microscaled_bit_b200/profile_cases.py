@@ -5,7 +5,9 @@ the 126 MB L2 but hold at most a few GB on the device.
   python -m mxfp4_microscaled_bit_b200.profile_cases --case gemm_prefill --iters 3
 cases: gemm_prefill (8192 x 14336 x 4096 NVFP4, 16-wide rotation), gemm_mxfp4,
 gemm_decode (16 x 14336 x 4096), quant_prefill (8192 x 4096 rotated, dynamic
-scale), kv_load (8 x 8 x 32768 x 128 cache to FP8), kv_store.
+scale), kv_load (8 x 8 x 32768 x 128 cache to FP8), kv_store, kv_attention (decode
+attention over the same 8 x 8 caches, G = 4), quant_mse (the 14336 x 4096 weight,
+MSE-optimal scales), gemm_quant (the prefill GEMM with its output NVFP4-encoded).
 """
 from __future__ import annotations
 
@@ -25,15 +27,29 @@ import synthetic_inputs as si  # noqa: E402
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
-                    choices=["gemm_prefill", "gemm_mxfp4", "gemm_decode", "quant_prefill", "kv_load", "kv_store"])
+                    choices=["gemm_prefill", "gemm_mxfp4", "gemm_decode", "quant_prefill", "kv_load", "kv_store",
+                             "kv_attention", "quant_mse", "gemm_quant"])
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if a.case in ("gemm_prefill", "gemm_mxfp4", "quant_prefill"):
+    if a.case == "quant_mse":
+        W = si.prefill_W().to(dev)
+        fn = lambda: fl.nvfp4_quantize(W, 16, mse=True)  # noqa: E731
+    elif a.case in ("gemm_prefill", "gemm_mxfp4", "quant_prefill", "gemm_quant"):
         A = si.prefill_A().to(dev)
         if a.case == "quant_prefill":
             fn = lambda: fl.nvfp4_quantize(A, 16)  # noqa: E731
+        elif a.case == "gemm_quant":
+            w = fl.prepare_weight(si.prefill_W().to(dev), "nvfp4", 16)
+            ca, sa, ga = fl.nvfp4_quantize(A, 16)
+            y = fl.nvfp4_gemm(ca, sa, ga, w.codes, w.scales, w.g)
+            _, _, gy = fl.nvfp4_quantize(y, 16)
+            del y
+            yc = torch.empty(A.shape[0], w.N // 2, dtype=torch.uint8, device=dev)
+            ys = torch.empty(fl.scale_bytes(A.shape[0], w.N // 16), dtype=torch.uint8, device=dev)
+            fn = lambda: fl.nvfp4_gemm_quant(ca, sa, ga, w.codes, w.scales, w.g, gy, hadamard=16,  # noqa: E731
+                                             write_y=False, y_codes=yc, y_scales=ys, workspace=False)
         else:
             fmt, had = ("nvfp4", 16) if a.case == "gemm_prefill" else ("mxfp4", 32)
             w = fl.prepare_weight(si.prefill_W().to(dev), fmt, had)
@@ -64,6 +80,12 @@ def main():
         if a.case == "kv_load":
             out = torch.empty(B, H, L, D, dtype=torch.uint8, device=dev)
             fn = lambda: fl.kv_nvfp4_load_fp8(codes, scales, g, L, out=out)  # noqa: E731
+        elif a.case == "kv_attention":
+            G = 4
+            q = si.normal_bf16(7, B * H * G, D).reshape(B, H * G, D).to(dev)
+            out = torch.empty(B, H * G, D, dtype=torch.float32, device=dev)
+            cache = (codes, scales, g)  # K and V: the same cache, read twice as K and as V
+            fn = lambda: fl.kv_nvfp4_attention(q, cache, cache, L, out=out)  # noqa: E731
         else:
             new = xd[:, :, :1].contiguous()
             pos = torch.full((B,), L - 1, dtype=torch.int32, device=dev)
