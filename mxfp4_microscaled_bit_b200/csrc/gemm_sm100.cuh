@@ -365,6 +365,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t *done_bar = acc_empty + C::NUM_ACC;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done_bar + 1);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *epi_ok = abort + 1;  // [2]: outcome of the accumulator wait, per tile parity
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -375,7 +376,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         for (int a = 0; a < C::NUM_ACC; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], C::EPI_WARPS * 32);
+            mbar_init(&acc_empty[a], C::EPI_WARPS);
         }
         mbar_init(done_bar, 1);
         *abort = 0;
@@ -520,7 +521,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tile_coords(p, w, mt, nt, sp);
             const int acc = it % C::NUM_ACC;
             const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
-            if (!warp_wait(&acc_full[acc], acc_phase, abort, lane))
+            // one warp waits on the accumulator; the others sleep in a named barrier (they issue
+            // nothing meanwhile, so the MMA-issuing warp keeps the SM's issue slots)
+            if (warp == 2) {
+                const bool okw = warp_wait(&acc_full[acc], acc_phase, abort, lane);
+                if (lane == 0)
+                    epi_ok[it & 1] = okw ? 1 : 0;
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(C::EPI_WARPS * 32) : "memory");
+            if (!epi_ok[it & 1])
                 break;
             tc_fence_after();
             float v[C::COLS_PER_WARP];
@@ -533,7 +542,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     tmem_ld32(taddr + c, v + c);
             }
             tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);  // accumulator free: the next tile's MMAs may start
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&acc_empty[acc]);  // this warp's part of the accumulator is free
 
             if constexpr (C::SWAP) {
                 // accumulator row = weight row n, column = activation row m: y[m, n]
