@@ -30,6 +30,7 @@ struct DeviceInfo {
     int sms = 0;
     bool gemm_attr[6] = {false, false, false, false, false, false};
     int pair_clusters[2] = {0, 0};  // resident clusters of the pair kernels (0: not yet queried)
+    bool attn_attr[KA_GMAX + 1] = {};  // dynamic shared memory raised for kv_attn_tc_kernel<G>
 };
 
 std::mutex g_mutex;
@@ -429,6 +430,22 @@ QuantShape make_shape(const void *x, int64_t rows, int64_t cols, int64_t ld_x, u
     return q;
 }
 
+template <int G>
+int launch_attn_tc(DeviceInfo *dev, dim3 grid, const KvAttnShape &a, cudaStream_t s)
+{
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (!dev->attn_attr[G]) {
+            if (cudaFuncSetAttribute(kv_attn_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     ka_tc_smem(G)) != cudaSuccess)
+                return FP4LIN_ERR_CUDA;
+            dev->attn_attr[G] = true;
+        }
+    }
+    kv_attn_tc_kernel<G><<<grid, KA_THREADS, ka_tc_smem(G), s>>>(a);
+    return launch_status();
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -650,15 +667,19 @@ int kv_nvfp4_attention(const void *q, const uint8_t *k_codes, const uint8_t *k_s
     a.S = (int)((L + KA_CHUNK - 1) / KA_CHUNK);
     const dim3 grid((unsigned)a.S, (unsigned)(B * H));
     cudaStream_t s = as_stream(stream);
-    switch (G) {
-    case 1: kv_attn_split_kernel<1><<<grid, KA_THREADS, 0, s>>>(a); break;
-    case 2: kv_attn_split_kernel<2><<<grid, KA_THREADS, 0, s>>>(a); break;
-    case 3: kv_attn_split_kernel<3><<<grid, KA_THREADS, 0, s>>>(a); break;
-    case 4: kv_attn_split_kernel<4><<<grid, KA_THREADS, 0, s>>>(a); break;
-    case 5: kv_attn_split_kernel<5><<<grid, KA_THREADS, 0, s>>>(a); break;
-    case 6: kv_attn_split_kernel<6><<<grid, KA_THREADS, 0, s>>>(a); break;
-    case 7: kv_attn_split_kernel<7><<<grid, KA_THREADS, 0, s>>>(a); break;
-    default: kv_attn_split_kernel<8><<<grid, KA_THREADS, 0, s>>>(a); break;
+    {
+        switch (G) {
+        case 1: st = launch_attn_tc<1>(dev, grid, a, s); break;
+        case 2: st = launch_attn_tc<2>(dev, grid, a, s); break;
+        case 3: st = launch_attn_tc<3>(dev, grid, a, s); break;
+        case 4: st = launch_attn_tc<4>(dev, grid, a, s); break;
+        case 5: st = launch_attn_tc<5>(dev, grid, a, s); break;
+        case 6: st = launch_attn_tc<6>(dev, grid, a, s); break;
+        case 7: st = launch_attn_tc<7>(dev, grid, a, s); break;
+        default: st = launch_attn_tc<8>(dev, grid, a, s); break;
+        }
+        if (st != FP4LIN_OK)
+            return st;
     }
     if (launch_status() != FP4LIN_OK)
         return FP4LIN_ERR_CUDA;

@@ -12,13 +12,13 @@
 //
 // Split over L (flash-decoding): CTA (s, bh) takes positions [s*chunk,
 // min(L, (s+1)*chunk)) of kv head bh for all G query heads (each K/V byte is
-// read once per group).  Pass 1: one thread per position forms the G scores
-// (q from shared memory, broadcast reads).  Pass 2: a half-warp per position,
-// lane l of a half owns dimensions 8l..8l+7.  The chunk's maximum, sum and unnormalised
-// output go to the workspace; kv_attn_merge_kernel combines the chunks.
+// read once per group), staging the chunk in shared memory with bulk async
+// copies; scores and the weighted sum of values run on the tensor cores
+// (kv_attn_tc_kernel).  The chunk's maximum, sum and unnormalised output go to
+// the workspace; kv_attn_merge_kernel combines the chunks.
 #pragma once
 
-#include "common.cuh"
+#include "gemm_sm100.cuh"  // mbarrier, bulk-copy and bounded-wait helpers
 
 namespace fp4lin {
 
@@ -27,6 +27,14 @@ constexpr int KA_THREADS = 256;
 constexpr int KA_WARPS = KA_THREADS / 32;
 constexpr int KA_CHUNK = 512;      // positions per CTA
 constexpr int KA_GMAX = 8;         // query heads per kv head
+constexpr int KA_SBUF = KA_CHUNK > KA_WARPS * KA_D ? KA_CHUNK : KA_WARPS * KA_D;  // score / output floats per head
+
+// Dynamic shared memory of kv_attn_tc_kernel<G>: the chunk's K and V codes and scales, the
+// score buffer, two mbarriers and an abort flag.
+constexpr int ka_tc_smem(int G)
+{
+    return KA_CHUNK * (KA_D / 2) * 2 + KA_CHUNK * (KA_D / 16) * 2 + KA_SBUF * G * 4 + 2 * 8 + 16;
+}
 
 struct KvAttnShape {
     const __nv_bfloat16 *q;        // [B, H*G, D]
@@ -79,89 +87,164 @@ __device__ __forceinline__ float2 half2_to_float2(uint32_t h)
                        __half2float(__ushort_as_half((unsigned short)(h >> 16))));
 }
 
-template <int G>
-__global__ void __launch_bounds__(KA_THREADS) kv_attn_split_kernel(KvAttnShape a)
+// ------------------------------------------------------------------ tensor-core form
+// D[16 x 8] += A[16 x 16] B[16 x 8], f16 operands, binary32 accumulation (the warp-level
+// MMA: one side of these products is at most 8 query heads, too small for tcgen05).
+// Fragments, with g = lane / 4, t = lane % 4: a0 = A[g][2t, 2t+1], a1 = A[g+8][2t, 2t+1],
+// a2 = A[g][2t+8, 2t+9], a3 = A[g+8][2t+8, 2t+9]; b0 = B[2t, 2t+1][g], b1 = B[2t+8, 2t+9][g];
+// d0, d1 = D[g][2t, 2t+1], d2, d3 = D[g+8][2t, 2t+1].
+__device__ __forceinline__ void mma_16816x(float *d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                           uint32_t b1)
 {
-    __shared__ __align__(16) float s_q[G * KA_D];
-    // pass 1: scores [chunk][G]; after pass 2: the warps' partial outputs [warps][G][D]
-    __shared__ __align__(16) float s_buf[(KA_CHUNK > KA_WARPS * KA_D ? KA_CHUNK : KA_WARPS * KA_D) * G];
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// f16x2 bit pattern of two floats (round to nearest).
+__device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi)
+{
+    return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
+}
+
+// Halves (lo of x, lo of y) or (hi of x, hi of y) of two f16x2 words.
+__device__ __forceinline__ uint32_t prmt_lo(uint32_t x, uint32_t y)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(x), "r"(y));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt_hi(uint32_t x, uint32_t y)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(x), "r"(y));
+    return r;
+}
+
+// Tensor-core form of the split kernel (same workspace output).  The CTA first stages its
+// chunk in shared memory: the K and V code rows (contiguous per kv head) by one bulk async
+// copy each, the scale rows by cooperative 8-byte loads, so every byte of the chunk is in
+// flight at once and V arrives while pass 1 runs.
+// Pass 1: scores^T by mma_16816x, A = K (16 positions as rows), B = q^T (8 heads as columns,
+// G used), one 16-dimension slice per MMA.  A common permutation of the dimensions leaves
+// the dot products unchanged; it is chosen so that a lane converts whole 32-bit code words:
+// word 4r + t (dimensions 32r + 8t .. +7) feeds slice 2r with its first four dimensions and
+// slice 2r+1 with its last four, and q is loaded in the same order.
+// Pass 2: o += p v by mma_16816x, A = the weights of 16 positions for 8 heads in rows 0..7
+// and the f16 rounding of what the f16 weights leave out in rows 8..15 (so p keeps ~22
+// bits and one MMA accumulates both), B = V with the output dimensions permuted so that a
+// lane needs 16 contiguous dimensions (8 code bytes, one scale) of each of its 4 rows; prmt
+// pairs two rows' values into one fragment register.
+template <int G>
+__global__ void __launch_bounds__(KA_THREADS, 2) kv_attn_tc_kernel(KvAttnShape a)
+{
+    extern __shared__ __align__(128) uint8_t ka_smem[];
+    uint8_t *s_kc = ka_smem;
+    uint8_t *s_vc = s_kc + KA_CHUNK * (KA_D / 2);
+    uint8_t *s_ks = s_vc + KA_CHUNK * (KA_D / 2);
+    uint8_t *s_vs = s_ks + KA_CHUNK * (KA_D / 16);
+    float *s_buf = reinterpret_cast<float *>(s_vs + KA_CHUNK * (KA_D / 16));  // [KA_SBUF * G]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(s_buf + KA_SBUF * G);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 2);
     __shared__ float s_red[KA_WARPS][G];
     __shared__ float s_m[G], s_sum[G];
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gq = lane >> 2, tg = lane & 3;
     const int64_t bh = blockIdx.y, b = bh / a.H, h = bh - b * a.H;
     const int64_t l0 = (int64_t)blockIdx.x * KA_CHUNK;
     const int n = (int)min((int64_t)KA_CHUNK, a.L - l0);
     const float kscale = __fmul_rn(__fmul_rn(*a.gk, 8.0f), 0.08838834764831845f);  // 8 g_k / sqrt(128)
-
-    const __nv_bfloat16 *qp = a.q + ((b * a.H + h) * G) * KA_D;
-    for (int i = tid; i < G * KA_D; i += KA_THREADS)
-        s_q[i] = __bfloat162float(qp[i]);
-    __syncthreads();
-
-    // ---- pass 1: scores, one thread per position
     const int64_t row0 = bh * a.Lcap + l0;
-    float mloc[G];
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const uint32_t bytes = (uint32_t)n * (KA_D / 2);  // a multiple of 64
+        mbar_expect_tx(&bars[0], bytes);
+        bulk_load(s_kc, a.kc + row0 * (KA_D / 2), bytes, &bars[0]);
+        mbar_expect_tx(&bars[1], bytes);
+        bulk_load(s_vc, a.vc + row0 * (KA_D / 2), bytes, &bars[1]);
+    }
+    for (int t = tid; t < n; t += KA_THREADS) {  // scale rows: 8-byte aligned only
+        *reinterpret_cast<uint2 *>(s_ks + t * 8) = ld_nc_v2(a.ks + (row0 + t) * (KA_D / 16));
+        *reinterpret_cast<uint2 *>(s_vs + t * 8) = ld_nc_v2(a.vs + (row0 + t) * (KA_D / 16));
+    }
+    // q^T as B fragments in the permuted dimension order (zero columns for heads >= G)
+    uint32_t qb[8][2];
 #pragma unroll
-    for (int j = 0; j < G; ++j)
-        mloc[j] = -INFINITY;
-    for (int t = tid; t < n; t += KA_THREADS) {
-        const uint8_t *crow = a.kc + (row0 + t) * (KA_D / 2);
-        const uint2 sc = ld_nc_v2(a.ks + (row0 + t) * (KA_D / 16));
-        float acc[G];
-#pragma unroll
-        for (int j = 0; j < G; ++j)
-            acc[j] = 0.0f;
-#pragma unroll
-        for (int hb = 0; hb < 4; ++hb) {  // 16 code bytes = two 16-value blocks
-            const uint4 cw = ld_nc_v4(crow + 16 * hb);
-            const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-            for (int wi = 0; wi < 4; ++wi) {
-                const int blk = 2 * hb + (wi >> 1);
-                const uint32_t sfb = ((blk < 4 ? sc.x : sc.y) >> (8 * (blk & 3))) & 0xFFu;
-                const uint32_t s2u = kv_scale_half2(sfb);
-                uint32_t hv[4];
-                kv_fp8_word(words[wi], s2u, hv);
-                float kv[8];
-#pragma unroll
-                for (int bi = 0; bi < 4; ++bi) {
-                    const float2 f = half2_to_float2(hv[bi]);
-                    kv[2 * bi] = f.x;
-                    kv[2 * bi + 1] = f.y;
-                }
-                const int d = 32 * hb + 8 * wi;  // the word's first dimension
-#pragma unroll
-                for (int j = 0; j < G; ++j) {
-                    const float4 q0 = *reinterpret_cast<const float4 *>(&s_q[j * KA_D + d]);
-                    const float4 q1 = *reinterpret_cast<const float4 *>(&s_q[j * KA_D + d + 4]);
-                    acc[j] = fmaf(q0.x, kv[0], acc[j]);
-                    acc[j] = fmaf(q0.y, kv[1], acc[j]);
-                    acc[j] = fmaf(q0.z, kv[2], acc[j]);
-                    acc[j] = fmaf(q0.w, kv[3], acc[j]);
-                    acc[j] = fmaf(q1.x, kv[4], acc[j]);
-                    acc[j] = fmaf(q1.y, kv[5], acc[j]);
-                    acc[j] = fmaf(q1.z, kv[6], acc[j]);
-                    acc[j] = fmaf(q1.w, kv[7], acc[j]);
-                }
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-            const float sj = __fmul_rn(acc[j], kscale);
-            s_buf[t * G + j] = sj;
-            mloc[j] = fmaxf(mloc[j], sj);
+    for (int r = 0; r < 4; ++r) {
+        if (gq < G) {
+            const uint4 u = ld_nc_v4(a.q + ((b * a.H + h) * G + gq) * KA_D + 32 * r + 8 * tg);
+            float f[8];
+            bf16x8_to_f32(u, f);
+            qb[2 * r][0] = f16x2_bits(f[0], f[1]);
+            qb[2 * r][1] = f16x2_bits(f[2], f[3]);
+            qb[2 * r + 1][0] = f16x2_bits(f[4], f[5]);
+            qb[2 * r + 1][1] = f16x2_bits(f[6], f[7]);
+        } else {
+            qb[2 * r][0] = qb[2 * r][1] = qb[2 * r + 1][0] = qb[2 * r + 1][1] = 0u;
         }
     }
-    // chunk maximum per query head
+    wait_bar(&bars[0], 0, abort);
+    __syncthreads();
+    const bool ok = *abort == 0;
+
+    // ---- pass 1: blocks of 16 positions; this lane loads positions t16 + gq and t16 + gq + 8
+    float mloc[2] = {-INFINITY, -INFINITY};  // heads 2tg, 2tg + 1
+    for (int t16 = warp * 16; ok && t16 < n; t16 += KA_WARPS * 16) {
+        const int pa = t16 + gq, pb = pa + 8;
+        uint32_t wa[4] = {0u, 0u, 0u, 0u}, wb[4] = {0u, 0u, 0u, 0u};
+        uint2 sa = make_uint2(0u, 0u), sb = make_uint2(0u, 0u);
+        if (pa < n) {
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-        float m = mloc[j];
+            for (int r = 0; r < 4; ++r)
+                wa[r] = *reinterpret_cast<const uint32_t *>(s_kc + pa * (KA_D / 2) + 4 * (4 * r + tg));
+            sa = *reinterpret_cast<const uint2 *>(s_ks + pa * 8);
+        }
+        if (pb < n) {
 #pragma unroll
-        for (int o = 16; o; o >>= 1)
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0)
-            s_red[warp][j] = m;
+            for (int r = 0; r < 4; ++r)
+                wb[r] = *reinterpret_cast<const uint32_t *>(s_kc + pb * (KA_D / 2) + 4 * (4 * r + tg));
+            sb = *reinterpret_cast<const uint2 *>(s_ks + pb * 8);
+        }
+        float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int blk = 2 * r + (tg >> 1);  // the block of dimensions 32r + 8t .. +7
+            const int sh = 8 * (blk & 3);
+            uint32_t ha[4], hb[4];
+            kv_fp8_word(wa[r], kv_scale_half2(((blk < 4 ? sa.x : sa.y) >> sh) & 0xFFu), ha);
+            kv_fp8_word(wb[r], kv_scale_half2(((blk < 4 ? sb.x : sb.y) >> sh) & 0xFFu), hb);
+            mma_16816x(sc, ha[0], hb[0], ha[1], hb[1], qb[2 * r][0], qb[2 * r][1]);
+            mma_16816x(sc, ha[2], hb[2], ha[3], hb[3], qb[2 * r + 1][0], qb[2 * r + 1][1]);
+        }
+        // sc[0], sc[1]: position pa, heads 2t, 2t+1; sc[2], sc[3]: position pb, same heads
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int hd = 2 * tg + (e & 1), pos = (e < 2) ? pa : pb;
+            if (hd < G && pos < n) {
+                const float sj = __fmul_rn(sc[e], kscale);
+                s_buf[pos * G + hd] = sj;
+                mloc[e & 1] = fmaxf(mloc[e & 1], sj);
+            }
+        }
+    }
+    // chunk maximum per head: the 8 lanes holding a head (same t), then the warps
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        float m = mloc[e];
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        if (gq == 0 && 2 * tg + e < G)
+            s_red[warp][2 * tg + e] = m;
     }
     __syncthreads();
     if (tid < G) {
@@ -171,12 +254,12 @@ __global__ void __launch_bounds__(KA_THREADS) kv_attn_split_kernel(KvAttnShape a
         s_m[tid] = m;
     }
     __syncthreads();
-    // weights p = exp(s - m) in place, and their sum per query head
+    // weights p = exp(s - m) in place, and their sum per head
     float sloc[G];
 #pragma unroll
     for (int j = 0; j < G; ++j)
         sloc[j] = 0.0f;
-    for (int t = tid; t < n; t += KA_THREADS)
+    for (int t = tid; ok && t < n; t += KA_THREADS)
 #pragma unroll
         for (int j = 0; j < G; ++j) {
             const float p = expf(s_buf[t * G + j] - s_m[j]);
@@ -192,60 +275,61 @@ __global__ void __launch_bounds__(KA_THREADS) kv_attn_split_kernel(KvAttnShape a
         if (lane == 0)
             s_red[warp][j] = sj;
     }
-    __syncthreads();
+    wait_bar(&bars[1], 0, abort);
+    __syncthreads();  // weights written, V landed
     if (tid < G) {
         float sj = 0.0f;
         for (int w = 0; w < KA_WARPS; ++w)
             sj += s_red[w][tid];
         s_sum[tid] = sj;
     }
+    const bool ok2 = *abort == 0;
 
-    // ---- pass 2: o = sum_l p_l v_l.  A warp takes two positions per step, a half-warp each;
-    // lane l of a half owns dimensions 8l..8l+7 (one 32-bit code word, scale byte l/2)
-    const int hl = lane & 15;
-    float o[G][8];
+    // ---- pass 2: blocks of 16 positions; n-tile u of the output holds dimension 16c + u in
+    // column c, so lane (gq, t) accumulates head gq at dimensions 32t + u and 32t + 16 + u
+    // (rows gq: the f16 weights' part, rows gq + 8: the rest's part)
+    float o[16][4];
 #pragma unroll
-    for (int j = 0; j < G; ++j)
+    for (int u = 0; u < 16; ++u)
+        o[u][0] = o[u][1] = o[u][2] = o[u][3] = 0.0f;
+    for (int t16 = warp * 16; ok2 && t16 < n; t16 += KA_WARPS * 16) {
+        const int rp[4] = {t16 + 2 * tg, t16 + 2 * tg + 1, t16 + 2 * tg + 8, t16 + 2 * tg + 9};
+        float p4[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            o[j][i] = 0.0f;
-    for (int t0 = 2 * warp; t0 < n; t0 += 2 * KA_WARPS) {
-        const int t = t0 + (lane >> 4);
-        if (t < n) {
-            const int64_t row = row0 + t;
-            const uint32_t w = *reinterpret_cast<const uint32_t *>(a.vc + row * (KA_D / 2) + 4 * hl);
-            const uint32_t s2u = kv_scale_half2(a.vs[row * (KA_D / 16) + (hl >> 1)]);
-            uint32_t hv[4];
-            kv_fp8_word(w, s2u, hv);
-            float v[8];
+        for (int e = 0; e < 4; ++e)
+            p4[e] = (gq < G && rp[e] < n) ? s_buf[rp[e] * G + gq] : 0.0f;
+        const uint32_t ah0 = f16x2_bits(p4[0], p4[1]), ah2 = f16x2_bits(p4[2], p4[3]);
+        const float2 b01 = half2_to_float2(ah0), b23 = half2_to_float2(ah2);
+        const uint32_t al0 = f16x2_bits(__fsub_rn(p4[0], b01.x), __fsub_rn(p4[1], b01.y));
+        const uint32_t al2 = f16x2_bits(__fsub_rn(p4[2], b23.x), __fsub_rn(p4[3], b23.y));
+        uint32_t hv[4][8];  // rows rp[0..3], dimensions 16gq + 2k, 2k + 1
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f = half2_to_float2(hv[k]);
-                v[2 * k] = f.x;
-                v[2 * k + 1] = f.y;
+        for (int e = 0; e < 4; ++e) {
+            uint2 c = make_uint2(0u, 0u);
+            uint32_t sfb = 0u;
+            if (rp[e] < n) {
+                c = *reinterpret_cast<const uint2 *>(s_vc + rp[e] * (KA_D / 2) + 8 * gq);
+                sfb = s_vs[rp[e] * 8 + gq];
             }
+            const uint32_t s2u = kv_scale_half2(sfb);
+            kv_fp8_word(c.x, s2u, hv[e]);
+            kv_fp8_word(c.y, s2u, hv[e] + 4);
+        }
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-                const float p = s_buf[t * G + j];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    o[j][i] = fmaf(p, v[i], o[j][i]);
-            }
+        for (int u = 0; u < 16; ++u) {
+            const int k = u >> 1;
+            const uint32_t b0 = (u & 1) ? prmt_hi(hv[0][k], hv[1][k]) : prmt_lo(hv[0][k], hv[1][k]);
+            const uint32_t b1 = (u & 1) ? prmt_hi(hv[2][k], hv[3][k]) : prmt_lo(hv[2][k], hv[3][k]);
+            mma_16816x(o[u], ah0, al0, ah2, al2, b0, b1);
         }
     }
-    // the two halves hold the same dimensions for different positions
-#pragma unroll
-    for (int j = 0; j < G; ++j)
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            o[j][i] += __shfl_xor_sync(0xffffffffu, o[j][i], 16);
     __syncthreads();  // every thread has read the weights: reuse s_buf for the warps' outputs
-    if (lane < 16)
+    if (gq < G)
 #pragma unroll
-        for (int j = 0; j < G; ++j)
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                s_buf[(warp * G + j) * KA_D + 8 * hl + i] = o[j][i];
+        for (int u = 0; u < 16; ++u) {
+            s_buf[(warp * G + gq) * KA_D + 32 * tg + u] = o[u][0] + o[u][2];
+            s_buf[(warp * G + gq) * KA_D + 32 * tg + 16 + u] = o[u][1] + o[u][3];
+        }
     __syncthreads();
     float *dst = a.ws + ((bh * a.S + blockIdx.x) * G) * (KA_D + 2);
     for (int i = tid; i < G * KA_D; i += KA_THREADS) {
