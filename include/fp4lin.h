@@ -280,6 +280,35 @@ int nvfp4_quantize_mse(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
 int mxfp4_quantize_nearest(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                            int hadamard, uint8_t *codes, uint8_t *scales, void *stream);
 
+/*
+ * Decode linear layer with the activation quantiser fused into the GEMM: the
+ * bf16 activations go straight in, and the GEMM's own warps encode each
+ * 16-row operand tile into shared memory as it is needed (the activations'
+ * online rotation and quantisation, MR-GPTQ abstract, "Abstract"; the native
+ * block-scaled FP4 product, "FP4 auf Blackwell", section "Was NVFP4 von
+ * frueheren 4-Bit-Formaten unterscheidet").  No codes or scales of the
+ * activations are written to memory and no quantiser is launched (one amax
+ * pass when the tensor scale is computed).  The result equals, bit for bit,
+ * nvfp4_quantize(x, hadamard, compute_global_scale, g_a) followed by
+ * nvfp4_gemm(codes, scales, g_a, w_codes, w_scales, g_w, y); with
+ * compute_global_scale = 1, *g_a is written with the same amax / 2688.
+ *   x: bf16 [M, K], row stride ld_x (multiple of 8 elements, 16-byte aligned);
+ *   w_codes / w_scales / g_w: the weights as nvfp4_gemm takes them (N x K);
+ *   y: bf16 [M, N], row stride ldy (multiple of 8).
+ * 1 <= M <= 16 (larger M: FP4LIN_ERR_UNSUPPORTED_SHAPE; use nvfp4_quantize +
+ * nvfp4_gemm), K a multiple of 64.  workspace: at least
+ * nvfp4_linear_decode_workspace_bytes(M, N, K) bytes (16-byte aligned): the
+ * amax partials, then the split-K partial sums; with less (or NULL, only
+ * allowed when compute_global_scale = 0) the GEMM runs without a K split.
+ * Errors as nvfp4_quantize and nvfp4_gemm.
+ */
+size_t nvfp4_linear_decode_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int hadamard,
+                        int compute_global_scale, float *g_a,
+                        const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w,
+                        void *y, int64_t N, int64_t ldy,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -27,7 +27,7 @@ __all__ = [
     "Fp4LinError", "lib", "nvfp4_quantize", "nvfp4_gemm", "mxfp4_quantize", "mxfp4_gemm",
     "kv_nvfp4_store", "kv_nvfp4_load_fp8", "scale_bytes", "gemm_workspace_bytes",
     "device_status", "convert_selftest", "QuantizedWeight", "prepare_weight", "nvfp4_linear",
-    "mxfp4_linear", "EXPORTS",
+    "mxfp4_linear", "nvfp4_linear_decode", "EXPORTS",
 ]
 
 STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA",
@@ -55,6 +55,9 @@ EXPORTS = {
                                   _sz, _vp]),
     "nvfp4_gemm_quant": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _vp, _vp, _vp, _i64, _i64, _i64,
                                 _vp, _sz, _vp]),
+    "nvfp4_linear_decode_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "nvfp4_linear_decode": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _sz,
+                                   _vp]),
 }
 
 _lock = threading.Lock()
@@ -238,6 +241,31 @@ def nvfp4_gemm_quant(a_codes, a_scales, g_a, w_codes, w_scales, g_w, g_y, *, had
     return y, y_codes, y_scales
 
 
+def nvfp4_linear_decode(x, w_codes, w_scales, g_w, *, hadamard: int = 0, g_a=None,
+                        compute_global_scale: bool | None = None, out=None, workspace=None, stream=None):
+    """Decode-sized (M <= 16) y = x W^T with the activation quantiser inside the GEMM: bit-equal to
+    nvfp4_quantize(x, hadamard, g_a, compute_global_scale=...) then nvfp4_gemm.  The activations'
+    tensor scale is computed (amax / 2688) when g_a is None or compute_global_scale is True (then
+    written into g_a), else taken from g_a.  Returns (y, g_a)."""
+    M, K = x.shape
+    N = w_codes.shape[0]
+    dev = x.device
+    y = _gemm_out(M, N, out, dev)
+    dynamic = (g_a is None) if compute_global_scale is None else bool(compute_global_scale)
+    if g_a is None:
+        g_a = torch.empty(1, dtype=torch.float32, device=dev)
+    if workspace is None:
+        need = lib().nvfp4_linear_decode_workspace_bytes(M, N, K)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    elif workspace is False:
+        workspace = None
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("nvfp4_linear_decode", lib().nvfp4_linear_decode(
+        _ptr(x), M, K, x.stride(0), hadamard, int(dynamic), _ptr(g_a), _ptr(w_codes), _ptr(w_scales), _ptr(g_w),
+        _ptr(y), N, y.stride(0), _ptr(workspace), wsb, _stream(stream)))
+    return y, g_a
+
+
 def mxfp4_gemm(a_codes, a_scales, w_codes, w_scales, *, out=None, workspace=None, stream=None):
     """y [M, N] bf16 = A_q W_q^T for MXFP4 operands."""
     M, K = a_codes.shape[0], a_codes.shape[1] * 2
@@ -306,7 +334,10 @@ def prepare_weight(w: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0) -> Qu
 
 
 def nvfp4_linear(x: torch.Tensor, w: QuantizedWeight, *, out=None, stream=None) -> torch.Tensor:
-    """y = x W^T: online (rotated) NVFP4 quantisation of x, then the block-scaled GEMM."""
+    """y = x W^T: online (rotated) NVFP4 quantisation of x, then the block-scaled GEMM (for M <= 16
+    one fused launch that quantises inside the GEMM; the same result)."""
+    if x.shape[0] <= 16 and x.shape[1] % 64 == 0:
+        return nvfp4_linear_decode(x, w.codes, w.scales, w.g, hadamard=w.hadamard, out=out, stream=stream)[0]
     c, s, g = nvfp4_quantize(x, w.hadamard, stream=stream)
     return nvfp4_gemm(c, s, g, w.codes, w.scales, w.g, out=out, stream=stream)
 

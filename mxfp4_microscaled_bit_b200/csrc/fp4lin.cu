@@ -28,7 +28,7 @@ struct DeviceInfo {
     bool probed = false;
     int status = FP4LIN_OK;
     int sms = 0;
-    bool gemm_attr[6] = {false, false, false, false, false, false};
+    bool gemm_attr[7] = {false, false, false, false, false, false, false};
     int pair_clusters[2] = {0, 0};  // resident clusters of the pair kernels (0: not yet queried)
     bool attn_attr[KA_GMAX + 1] = {};  // dynamic shared memory raised for kv_attn_tc_kernel<G>
 };
@@ -195,11 +195,21 @@ int raster_group(int num_mt)
     return std::max(1, std::min(g, num_mt));
 }
 
+// The bf16 activations a fused decode GEMM quantises itself (GemmCfg FUSEQ).
+struct FuseIn {
+    const void *x;
+    int64_t ld;
+    int had;
+    const float *part;  // amax partials (npart > 0: dynamic tensor scale, written to g_out)
+    int npart;
+    float *g_out;
+};
+
 template <class C>
 int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const uint8_t *a_codes,
                     const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes, const uint8_t *w_scales,
                     const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy, float *ws,
-                    cudaStream_t st, const QuantOut &qo)
+                    cudaStream_t st, const QuantOut &qo, const FuseIn *fi = nullptr)
 {
     {
         std::lock_guard<std::mutex> lk(g_mutex);
@@ -211,7 +221,11 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
         }
     }
     CUtensorMap tmA, tmB;
-    if (!make_code_map(&tmA, a_codes, M, K, 128) || !make_code_map(&tmB, w_codes, N, K, C::BN))
+    if (!make_code_map(&tmA, a_codes, M, K, 128))
+        return FP4LIN_ERR_CUDA;
+    if (fi)
+        tmB = tmA;  // not used: the kernel quantises the activations itself
+    else if (!make_code_map(&tmB, w_codes, N, K, C::BN))
         return FP4LIN_ERR_CUDA;
     GemmParams p{};
     p.sfa = a_scales;
@@ -238,6 +252,14 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
     p.qg = qo.qg;
     p.qhad = qo.qhad;
     p.qkatoms = qo.qkatoms;
+    if (fi) {
+        p.xa = reinterpret_cast<const __nv_bfloat16 *>(fi->x);
+        p.ld_xa = fi->ld;
+        p.xhad = fi->had;
+        p.xpart = fi->part;
+        p.xnpart = fi->npart;
+        p.g_a_out = fi->g_out;
+    }
     const int grid = (int)std::min<int64_t>(p.work, dev->sms);
     fp4_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, p);
     if (launch_status() != FP4LIN_OK)
@@ -685,6 +707,71 @@ int kv_nvfp4_attention(const void *q, const uint8_t *k_codes, const uint8_t *k_s
         return FP4LIN_ERR_CUDA;
     kv_attn_merge_kernel<<<(unsigned)((int64_t)B * H * G), KA_D, 0, s>>>(a, G);
     return launch_status();
+}
+
+size_t nvfp4_linear_decode_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 1 || M > 16 || N < 1 || K < 64)
+        return 0;
+    int sms = 148, dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            sms = v;
+    } else {
+        cudaGetLastError();
+    }
+    return AMAX_MAX_BLOCKS * sizeof(float) + plan_decode(M, N, K, sms).ws_bytes;
+}
+
+int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int hadamard, int compute_global_scale,
+                        float *g_a, const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w, void *y,
+                        int64_t N, int64_t ldy, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!x || !g_a || !w_codes || !w_scales || !g_w || !y)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (M < 1 || N < 1 || K < 1 || ld_x < K || ldy < N || (hadamard != 0 && hadamard != 16) ||
+        (compute_global_scale != 0 && compute_global_scale != 1))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (M > 16 || K % 64 != 0 || ld_x % 8 != 0 || ldy % 8 != 0 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(x, 16) || !aligned(w_codes, 16) || !aligned(w_scales, 16) || !aligned(y, 16) || !aligned(g_a, 4) ||
+        !aligned(g_w, 4) || (workspace && !aligned(workspace, 16)))
+        return FP4LIN_ERR_MISALIGNED;
+    if (compute_global_scale && (!workspace || workspace_bytes < AMAX_MAX_BLOCKS * sizeof(float)))
+        return FP4LIN_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    cudaStream_t s = as_stream(stream);
+    GemmPlan pl = plan_decode(M, N, K, dev->sms);
+    float *part = reinterpret_cast<float *>(workspace);
+    float *ws = nullptr;
+    const size_t ws_have = workspace_bytes > AMAX_MAX_BLOCKS * sizeof(float)
+                               ? workspace_bytes - AMAX_MAX_BLOCKS * sizeof(float) : 0;
+    if (pl.splits > 1 && (!workspace || ws_have < pl.ws_bytes)) {  // no room for partial sums: run unsplit
+        pl.splits = 1;
+        pl.kps = pl.nk;
+    }
+    if (pl.splits > 1)
+        ws = part + AMAX_MAX_BLOCKS;
+    FuseIn fi{x, ld_x, hadamard, nullptr, 0, g_a};
+    if (compute_global_scale) {
+        QuantShape q = make_shape(x, M, K, ld_x, nullptr, nullptr, 16);
+        const dim3 agrid = amax_grid(q);
+        fi.part = part;
+        fi.npart = (int)(agrid.x * agrid.y);
+        if (hadamard)
+            nvfp4_amax_kernel<true><<<agrid, QTHREADS, 0, s>>>(q, part);
+        else
+            nvfp4_amax_kernel<false><<<agrid, QTHREADS, 0, s>>>(q, part);
+        if (launch_status() != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+    }
+    // swapped form: the weights are the MMA's M side; g_w's slot carries the activations' scale
+    return launch_gemm_cfg<GemmCfg<16, true, true, true>>(dev, 6, pl, w_codes, w_scales, g_w, nullptr, nullptr, g_a,
+                                                           y, N, M, K, ldy, ws, s, QuantOut{}, &fi);
 }
 
 int nvfp4_gemm_quant(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,

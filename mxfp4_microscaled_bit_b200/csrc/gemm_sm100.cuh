@@ -218,11 +218,15 @@ __device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr)
 // SWAP: the MMA computes y^T = W A^T -- its M operand is W (128 rows per tile), its N
 // operand the few activation rows (BN = 16) -- and the epilogue writes y transposed.  For
 // decode-sized M every tile then streams 128 weight rows instead of padding M to 128.
-template <int BN_, bool NV_, bool SWAP_ = false>
+// FUSEQ (decode, with SWAP): the activations arrive as bf16 and the epilogue warps quantise
+// them into each stage themselves (NVFP4, the quantiser's arithmetic), instead of TMA loading
+// codes and scales a separate quantiser wrote.
+template <int BN_, bool NV_, bool SWAP_ = false, bool FUSEQ_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool NV = NV_;                       // NVFP4 (16-blocks, E4M3) or MXFP4 (32-blocks, E8M0)
     static constexpr bool SWAP = SWAP_;
+    static constexpr bool FUSEQ = FUSEQ_;
     static constexpr int BM = 128;
     static constexpr int BK = 256;                        // elements per stage (128 code bytes per row)
     static constexpr int MMA_K = 64;
@@ -252,6 +256,7 @@ struct GemmCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory overflow");
     static_assert(STAGES >= 2, "pipeline too shallow");
     static_assert(!SWAP || BN == 16, "the swapped form serves at most 16 activation rows");
+    static_assert(!FUSEQ || (SWAP && NV), "the fused activation quantiser is the NVFP4 decode form's");
     static_assert(SWAP || COLS_PER_WARP % 32 == 0, "epilogue loads 32 columns at a time");
 };
 
@@ -272,6 +277,16 @@ struct GemmParams {
     const float *qg;
     int qhad;
     int64_t qkatoms;
+    // FUSEQ: the bf16 activations [p.N rows, K] (row stride ld_xa), rotated by H_16/4 when
+    // xhad; their tensor scale is *g_w (static; the swapped form's activation slot) or, when
+    // xnpart > 0, amax / 2688 over the xnpart partial maxima at xpart, written to g_a_out by
+    // CTA 0.
+    const __nv_bfloat16 *xa;
+    int64_t ld_xa;
+    int xhad;
+    const float *xpart;
+    int xnpart;
+    float *g_a_out;
 };
 
 // NVFP4-encode 16 consecutive output values of one row held by this thread (already
@@ -351,6 +366,55 @@ __device__ __forceinline__ void tile_coords(const GemmParams &p, int64_t w, int 
     nt = (int)(idx / rows);
 }
 
+// FUSEQ: one epilogue thread (et = 0..255) owns activation block (row et / 16, block et % 16)
+// of every k-tile.  fuseq_load fetches its 16 bf16 values (nothing outside the activations);
+// fuseq_store quantises them into the stage: the 8 code bytes at their place in the
+// 128-byte-swizzled 16-row operand tile (16-byte chunk index XOR row % 8), the scale byte at
+// its place in the stage's scale atoms; blocks outside the activations get zeros.  The same
+// arithmetic as nvfp4_quant_kernel, so the codes and scales are those it would write.
+struct FuseRaw {
+    uint4 u0, u1;
+};
+
+__device__ __forceinline__ bool fuseq_valid(const GemmParams &p, int kt, int et)
+{
+    return (et >> 4) < p.N && (int64_t)kt * 256 + 16 * (et & 15) < p.K;
+}
+
+__device__ __forceinline__ void fuseq_load(const GemmParams &p, int kt, int et, FuseRaw &r)
+{
+    if (fuseq_valid(p, kt, et)) {
+        const __nv_bfloat16 *src = p.xa + (et >> 4) * p.ld_xa + (int64_t)kt * 256 + 16 * (et & 15);
+        r.u0 = ld_nc_v4(src);
+        r.u1 = ld_nc_v4(src + 8);
+    }
+}
+
+__device__ __forceinline__ void fuseq_store(const GemmParams &p, uint8_t *sB, uint8_t *sSFB, int kt, int et,
+                                            const FuseRaw &x, float xg)
+{
+    const int r = et >> 4, c = et & 15;
+    uint32_t lo = 0u, hi = 0u, sf = 0u;
+    if (fuseq_valid(p, kt, et)) {
+        const uint32_t raw[8] = {x.u0.x, x.u0.y, x.u0.z, x.u0.w, x.u1.x, x.u1.y, x.u1.z, x.u1.w};
+        float v[16];
+        if (p.xhad)
+            nvfp4_block_values<true>(raw, v);
+        else
+            nvfp4_block_values<false>(raw, v);
+        float rcp;
+        sf = nvfp4_block_scale(abs_max<16>(v), xg, rcp);
+        scale_packed<16>(v, rcp);
+        lo = pack_e2m1x8(v);
+        hi = pack_e2m1x8(v + 8);
+    }
+    *reinterpret_cast<uint2 *>(sB + r * 128 + (((c >> 1) ^ (r & 7)) << 4) + ((c & 1) << 3)) = make_uint2(lo, hi);
+    sSFB[(c >> 2) * 512 + r * 16 + (c & 3)] = (uint8_t)sf;
+}
+
+// k-tiles whose activations are fetched ahead of the one being encoded
+constexpr int FUSEQ_PREFETCH = 3;
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmParams p)
@@ -371,7 +435,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], C::FUSEQ ? 1 + C::EPI_WARPS : 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < C::NUM_ACC; ++a) {
@@ -380,6 +444,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         mbar_init(done_bar, 1);
         *abort = 0;
+        epi_ok[2] = 0;  // the epilogue warps' failure flag
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
@@ -414,17 +479,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     uint8_t *sB = sA + C::A_BYTES;
                     uint8_t *sSFA = sB + C::B_BYTES;
                     uint8_t *sSFB = sSFA + C::SFA_BYTES;
-                    mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + C::RT));
+                    if constexpr (C::FUSEQ)  // the activation half of the stage comes from the epilogue warps
+                        mbar_expect_tx(&full[stage], C::A_BYTES + atoms * 512);
+                    else
+                        mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + C::RT));
                     armed |= 1u << stage;
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
                     tma_load_2d(sA, &tmA, &full[stage], kt * 128, mt * C::BM);
-                    tma_load_2d(sB, &tmB, &full[stage], kt * 128, nt * C::BN);
                     const int64_t ka = (int64_t)kt * C::APK;
                     bulk_load(sSFA, p.sfa + ((int64_t)mt * p.katoms + ka) * 512, atoms * 512, &full[stage]);
+                    if constexpr (!C::FUSEQ) {
+                        tma_load_2d(sB, &tmB, &full[stage], kt * 128, nt * C::BN);
 #pragma unroll
-                    for (int rt = 0; rt < C::RT; ++rt)
-                        bulk_load(sSFB + rt * C::APK * 512, p.sfb + ((brt0 + rt) * p.katoms + ka) * 512, atoms * 512,
-                                  &full[stage]);
+                        for (int rt = 0; rt < C::RT; ++rt)
+                            bulk_load(sSFB + rt * C::APK * 512, p.sfb + ((brt0 + rt) * p.katoms + ka) * 512,
+                                      atoms * 512, &full[stage]);
+                    }
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -514,11 +584,105 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ---------------------------------------------------------------- epilogue
         const int quad = warp & 3;                       // TMEM lanes this warp may access
         const int half = (warp - 2) >> 2;                // which half of the tile's columns
-        const float gg = C::NV ? __fmul_rn(*p.g_a, *p.g_w) : 1.0f;
+        const int et = threadIdx.x - 64;                 // 0..255 over the epilogue warps
+        float gg = C::NV ? __fmul_rn(*p.g_a, *p.g_w) : 1.0f;
+        float xg = 0.0f;                                 // FUSEQ: the activations' tensor scale
+        __shared__ float s_xred[C::EPI_WARPS];
+        __shared__ float s_xg;
+        if constexpr (C::FUSEQ) {
+            if (p.xnpart > 0) {  // amax over the partial maxima, reduced in a fixed order
+                float m = 0.0f;
+                for (int k = et; k < p.xnpart; k += C::EPI_WARPS * 32)
+                    m = fmaxf(m, p.xpart[k]);
+#pragma unroll
+                for (int o = 16; o; o >>= 1)
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+                if (lane == 0)
+                    s_xred[warp - 2] = m;
+                asm volatile("bar.sync 1, %0;" ::"r"(C::EPI_WARPS * 32) : "memory");
+                if (et == 0) {
+                    float b = 0.0f;
+                    for (int k = 0; k < C::EPI_WARPS; ++k)
+                        b = fmaxf(b, s_xred[k]);
+                    float g = __fdiv_rn(b, 2688.0f);  // 6 * 448, as the quantiser
+                    if (!(g > 0.0f))
+                        g = 1.0f;
+                    s_xg = g;
+                    if (blockIdx.x == 0)
+                        *p.g_a_out = g;
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(C::EPI_WARPS * 32) : "memory");
+                xg = s_xg;
+            } else {
+                xg = *p.g_w;  // swapped form: g_w is the activations' slot, g_a the weights'
+            }
+            gg = __fmul_rn(xg, *p.g_a);
+            // scale-atom rows past the 16 activation rows: zero once in every stage
+            for (int s = 0; s < C::STAGES; ++s) {
+                uint8_t *sfb = smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES + C::SFA_BYTES;
+                for (int i = et; i < C::SFB_BYTES / 16; i += C::EPI_WARPS * 32)
+                    *reinterpret_cast<uint4 *>(sfb + 16 * i) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"r"(C::EPI_WARPS * 32) : "memory");  // zeros before any fill
+        }
+        volatile int *epi_fail = epi_ok + 2;
+        int qstage = 0;
+        uint32_t qphase = 0;
+        // FUSEQ: fill the activation operand of item w's stages, as the producer fills the
+        // weights; the k-tile's values are fetched FUSEQ_PREFETCH k-tiles ahead of their encoding.
+        // Returns false (all epilogue warps agree) when a wait gave up.
+        auto fill_item = [&](int64_t w) -> bool {
+            int mt, nt, sp;
+            tile_coords(p, w, mt, nt, sp);
+            const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+            FuseRaw buf[FUSEQ_PREFETCH];
+#pragma unroll
+            for (int j = 0; j < FUSEQ_PREFETCH; ++j)
+                if (kt0 + j < kt1)
+                    fuseq_load(p, kt0 + j, et, buf[j]);
+            bool okq = true;
+            for (int base = kt0; okq && base < kt1; base += FUSEQ_PREFETCH) {
+#pragma unroll
+                for (int j = 0; j < FUSEQ_PREFETCH; ++j) {
+                    const int kt = base + j;
+                    if (kt >= kt1)
+                        break;
+                    const FuseRaw cur = buf[j];
+                    if (kt + FUSEQ_PREFETCH < kt1)
+                        fuseq_load(p, kt + FUSEQ_PREFETCH, et, buf[j]);
+                    if (!(okq = warp_wait(&empty[qstage], qphase ^ 1u, abort, lane)))
+                        break;
+                    uint8_t *sB = smem + qstage * C::STAGE_BYTES + C::A_BYTES;
+                    fuseq_store(p, sB, sB + C::B_BYTES + C::SFA_BYTES, kt, et, cur, xg);
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&full[qstage]);
+                    if (++qstage == C::STAGES) {
+                        qstage = 0;
+                        qphase ^= 1u;
+                    }
+                }
+            }
+            if (!okq && lane == 0)
+                *epi_fail = 1;
+            asm volatile("bar.sync 1, %0;" ::"r"(C::EPI_WARPS * 32) : "memory");  // agree before going on
+            return *epi_fail == 0;
+        };
+        if constexpr (C::FUSEQ) {
+            if (blockIdx.x < p.work)
+                (void)fill_item(blockIdx.x);
+        }
         int it = 0;
         for (int64_t w = blockIdx.x; w < p.work; w += gridDim.x, ++it) {
             int mt, nt, sp;
             tile_coords(p, w, mt, nt, sp);
+            if constexpr (C::FUSEQ) {
+                // the next item's operand first, so its MMAs can start while this item drains
+                if (*epi_fail || (w + gridDim.x < p.work && !fill_item(w + gridDim.x)))
+                    break;
+            }
             const int acc = it % C::NUM_ACC;
             const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
             // one warp waits on the accumulator; the others sleep in a named barrier (they issue

@@ -23,7 +23,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported():
     names = header_functions()
-    assert len(names) == 18, names
+    assert len(names) == 20, names
     L = fl.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -108,7 +108,30 @@ def test_kv_argument_checks():
     assert L.fp4lin_convert_selftest(P, P, P, 0, None) == INVALID
 
 
+def d(M=16, K=128, ldx=128, had=0, dyn=0, ga=P, x=P, y=P, N=64, ldy=64, ws=P, wsb=8192):
+    return fl.lib().nvfp4_linear_decode(x, M, K, ldx, had, dyn, ga, P, P, P, y, N, ldy, ws, wsb, None)
+
+
+def test_linear_decode_argument_checks():
+    assert d(x=None) == INVALID
+    assert d(ga=None) == INVALID
+    assert d(M=0) == INVALID
+    assert d(had=32) == INVALID
+    assert d(dyn=3) == INVALID
+    assert d(ldx=64) == INVALID
+    assert d(M=17) == SHAPE  # decode sizes only
+    assert d(K=96, ldx=96) == SHAPE
+    assert d(ldy=68, N=66) == SHAPE
+    assert d(x=P + 8) == MISALIGNED
+    assert d(dyn=1, ws=None) == WORKSPACE
+    assert d(dyn=1, wsb=1000) == WORKSPACE
+    L = fl.lib()
+    assert L.nvfp4_linear_decode_workspace_bytes(17, 64, 128) == 0
+    assert L.nvfp4_linear_decode_workspace_bytes(16, 4096, 4096) >= 4096
+
+
 @pytest.mark.parametrize("fn", ["nvfp4_quantize", "mxfp4_quantize", "nvfp4_gemm", "mxfp4_gemm",
-                                "kv_nvfp4_store", "kv_nvfp4_load_fp8"])
+                                "kv_nvfp4_store", "kv_nvfp4_load_fp8", "nvfp4_linear_decode", "nvfp4_gemm_quant",
+                                "kv_nvfp4_attention"])
 def test_binding_names_match_abi(fn):
     assert callable(getattr(fl, fn))
