@@ -149,8 +149,9 @@ class Workload:
         self.A_host = si.prefill_A().pin_memory()
         W = si.prefill_W()
         self.A = self.A_host.to(dev)
-        self.w = fl.prepare_weight(W.to(dev), "nvfp4", hadamard=16)  # offline: rotated + quantised once
-        self.w_mx = fl.prepare_weight(W.to(dev), "mxfp4", hadamard=32)
+        self.W_bf16 = W.to(dev)  # kept for the bf16 context number
+        self.w = fl.prepare_weight(self.W_bf16, "nvfp4", hadamard=16)  # offline: rotated + quantised once
+        self.w_mx = fl.prepare_weight(self.W_bf16, "mxfp4", hadamard=32)
         del W
         M, K = self.M, self.K
         self.a_codes = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
@@ -259,6 +260,56 @@ class Workload:
         self.fl.nvfp4_gemm_quant(self.a_codes, self.a_scales, self.g_a, self.w.codes, self.w.scales, self.w.g,
                                  self.g_y, hadamard=16, write_y=False, y_codes=self.y_codes,
                                  y_scales=self.y_scales, workspace=False)
+
+    def decode_setup(self, M=16, N=14336, K=4096, hadamard=0):
+        """The decode linear layer (M activation rows, dynamic tensor scale) as two CUDA
+        graphs of `copies` calls each, every call against its own copy of the weights (together
+        larger than L2, so each call streams its weights from HBM): quantise then GEMM, and the
+        GEMM that quantises the activations itself.  -> (unfused, fused, calls per replay)."""
+        fl, dev = self.fl, self.dev
+        w0 = fl.prepare_weight(si.decode_W(N, K).to(dev), "nvfp4", hadamard)
+        copies = int(300e6 // (N * K * (0.5 + 1 / 16))) + 1
+        Ws = [(w0.codes.clone(), w0.scales.clone(), w0.g.clone()) for _ in range(copies)]
+        x = si.decode_A(M, K).to(dev)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        g = torch.empty(1, dtype=torch.float32, device=dev)
+        c = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        sc = torch.empty(fl.scale_bytes(M, K // 16), dtype=torch.uint8, device=dev)
+        qws = torch.empty(1024, dtype=torch.float32, device=dev)
+        gws = torch.empty(max(16, fl.gemm_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+        dws = torch.empty(max(16, fl.lib().nvfp4_linear_decode_workspace_bytes(M, N, K)), dtype=torch.uint8,
+                          device=dev)
+
+        def unfused(st):
+            for wc, wsc, wg in Ws:
+                fl.nvfp4_quantize(x, hadamard, g, compute_global_scale=True, codes=c, scales=sc, workspace=qws,
+                                  stream=st)
+                fl.nvfp4_gemm(c, sc, g, wc, wsc, wg, out=y, workspace=gws, stream=st)
+
+        def fused(st):
+            for wc, wsc, wg in Ws:
+                fl.nvfp4_linear_decode(x, wc, wsc, wg, hadamard=hadamard, g_a=g, compute_global_scale=True, out=y,
+                                       workspace=dws, stream=st)
+
+        st = torch.cuda.Stream()
+        graphs = []
+        with torch.cuda.stream(st):
+            for fn in (unfused, fused):
+                fn(st)  # warm: kernel attributes set outside the capture
+                st.synchronize()
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=st):
+                    fn(st)
+                graphs.append(gr)
+        torch.cuda.synchronize()
+        self.decode_shape = (M, N, K)
+        self.decode_launches = {"unfused": 3 + (fl.gemm_workspace_bytes(M, N, K) > 0),
+                                "fused": 2 + (fl.lib().nvfp4_linear_decode_workspace_bytes(M, N, K) > 4096)}
+        return graphs[0].replay, graphs[1].replay, copies
+
+    def decode_bytes(self):
+        M, N, K = self.decode_shape
+        return N * K * (0.5 + 1 / 16) + M * K * 2 + M * N * 2  # weights once, bf16 x in, bf16 y out
 
     def attention_setup(self, G):
         """-> a callable running kv_nvfp4_attention over the decode step's caches."""
@@ -451,6 +502,25 @@ def main():
     fused_ms = time_loop(w.gemm_quant_fused, 20, stream) / 20
     assert fl.device_status() == 0
 
+    # ---- context: cuBLAS bf16 on the same prefill product (torch.matmul of the unquantised operands)
+    a_bf = w.A
+    w_bf = w.W_bf16
+    y_bf = torch.empty_like(w.y)
+    mm = lambda: torch.matmul(a_bf, w_bf.t(), out=y_bf)
+    for _ in range(3):
+        mm()
+    bf16_ms = time_loop(mm, 10, stream) / 10
+    del w_bf, y_bf
+
+    # ---- the decode linear layer: quantise then GEMM vs the GEMM that quantises its input
+    dec_unfused, dec_fused, dec_calls = w.decode_setup()
+    for _ in range(3):
+        dec_unfused()
+        dec_fused()
+    dec_unfused_us = time_loop(dec_unfused, 10, stream) / (10 * dec_calls) * 1e3
+    dec_fused_us = time_loop(dec_fused, 10, stream) / (10 * dec_calls) * 1e3
+    assert fl.device_status() == 0
+
     # ---- decode attention straight from the NVFP4 caches (G = 4 query heads per kv head)
     attn = w.attention_setup(4)
     for _ in range(3):
@@ -540,6 +610,10 @@ def main():
                     "kv_load_gbs": rooflines["kv_load_fp8"]["achieved"],
                     "kv_store_us": st_ms * 1e3,
                     "mxfp4_layer_tflops": flops / (mx_ms * 1e-3) / 1e12,
+                    "bf16_matmul_context": {"ms": bf16_ms, "tflops": flops / (bf16_ms * 1e-3) / 1e12,
+                                            "layer_speedup": bf16_ms / layer_ms, "gemm_speedup": bf16_ms / gemm_ms,
+                                            "note": "torch.matmul (cuBLAS) bf16 on the unquantised prefill "
+                                                    "operands, back-to-back calls"},
                     "kv_attention": {
                         "ms": attn_ms, "G": w.attn_G,
                         "gbs": w.attention_bytes() / (attn_ms * 1e-3) / 1e9,
@@ -548,6 +622,15 @@ def main():
                         "note": "decode attention over the NVFP4 caches with the FP8 values formed on chip; "
                                 "kv_load_fp8_ms is the step's FP8 load of the same caches, which an FP8 "
                                 "attention kernel would then read back"},
+                    "decode_layer": {
+                        "shape_mnk": list(w.decode_shape), "unfused_us": dec_unfused_us, "fused_us": dec_fused_us,
+                        "speedup": dec_unfused_us / dec_fused_us,
+                        "fused_gbs": w.decode_bytes() / (dec_fused_us * 1e-6) / 1e9,
+                        "fused_frac_hbm": w.decode_bytes() / (dec_fused_us * 1e-6) / 1e9 / hbm,
+                        "launches": w.decode_launches,
+                        "note": "decode config (no rotation), dynamic tensor scale; nvfp4_quantize + nvfp4_gemm vs "
+                                "nvfp4_linear_decode (amax pass + the GEMM that encodes its input + split-K "
+                                "reduction); CUDA-graph replay, each call on its own weight copy (> L2)"},
                     "next_layer_input": {
                         "gemm_then_quantize_ms": unfused_ms, "gemm_quant_fused_ms": fused_ms,
                         "speedup": unfused_ms / fused_ms,

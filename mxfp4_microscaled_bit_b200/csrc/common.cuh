@@ -23,6 +23,13 @@ __device__ __forceinline__ void report_error(unsigned int code)
 }
 
 // ------------------------------------------------------------------ loads
+// Programmatic dependent launch.  pdl_trigger: this CTA lets the next kernel in the stream
+// (launched with programmatic stream serialisation) start early.  pdl_wait: block until the
+// preceding kernel has completed and its writes are visible (returns at once when this
+// kernel was launched without the attribute).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint4 ld_nc_v4(const void *p)
 {
     uint4 r;

@@ -195,6 +195,25 @@ int raster_group(int num_mt)
     return std::max(1, std::min(g, num_mt));
 }
 
+// Launch with programmatic stream serialisation: the kernel may start before the previous one
+// in the stream has finished, and must pdl_wait before touching anything that one writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                       Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // The bf16 activations a fused decode GEMM quantises itself (GemmCfg FUSEQ).
 struct FuseIn {
     const void *x;
@@ -261,16 +280,26 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
         p.g_a_out = fi->g_out;
     }
     const int grid = (int)std::min<int64_t>(p.work, dev->sms);
-    fp4_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, p);
+    if (fi && fi->npart > 0) {  // overlaps the amax pass: only the activation encoders wait for it
+        if (launch_pdl(fp4_gemm_kernel<C>, grid, C::THREADS, C::SMEM_BYTES, st, tmA, tmB, p) != cudaSuccess) {
+            cudaGetLastError();
+            return FP4LIN_ERR_CUDA;
+        }
+    } else {
+        fp4_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, p);
+    }
     if (launch_status() != FP4LIN_OK)
         return FP4LIN_ERR_CUDA;
     if (pl.splits > 1) {
         const int64_t rM = C::SWAP ? N : M, rN = C::SWAP ? M : N;  // the output's shape
         const int64_t items = rM * ((rN + 3) / 4);
         const int rgrid = (int)std::min<int64_t>((items + 255) / 256, (int64_t)dev->sms * 8);
-        splitk_reduce_kernel<<<rgrid, 256, 0, st>>>(ws, pl.splits, rM, rN, pl.ldw, C::NV ? g_a : nullptr,
-                                                    C::NV ? g_w : nullptr, reinterpret_cast<__nv_bfloat16 *>(y),
-                                                    ldy, qo);
+        const float *ga = C::NV ? g_a : nullptr, *gw = C::NV ? g_w : nullptr;
+        if (launch_pdl(splitk_reduce_kernel, rgrid, 256, 0, st, (const float *)ws, pl.splits, rM, rN, pl.ldw, ga, gw,
+                       reinterpret_cast<__nv_bfloat16 *>(y), ldy, qo) != cudaSuccess) {
+            cudaGetLastError();
+            return FP4LIN_ERR_CUDA;
+        }
         if (launch_status() != FP4LIN_OK)
             return FP4LIN_ERR_CUDA;
     }
@@ -709,6 +738,12 @@ int kv_nvfp4_attention(const void *q, const uint8_t *k_codes, const uint8_t *k_s
     return launch_status();
 }
 
+// Up to this many activation values, every CTA of the fused decode GEMM computes their amax
+// itself rather than waiting for a separate amax pass.
+#ifndef FUSED_AMAX_MAX
+#define FUSED_AMAX_MAX 16384
+#endif
+
 size_t nvfp4_linear_decode_workspace_bytes(int64_t M, int64_t N, int64_t K)
 {
     if (M < 1 || M > 16 || N < 1 || K < 64)
@@ -757,7 +792,9 @@ int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int h
     if (pl.splits > 1)
         ws = part + AMAX_MAX_BLOCKS;
     FuseIn fi{x, ld_x, hadamard, nullptr, 0, g_a};
-    if (compute_global_scale) {
+    if (compute_global_scale && M * K <= FUSED_AMAX_MAX) {
+        fi.npart = -1;  // each CTA takes the amax itself: cheaper than a launch for so few values
+    } else if (compute_global_scale) {
         QuantShape q = make_shape(x, M, K, ld_x, nullptr, nullptr, 16);
         const dim3 agrid = amax_grid(q);
         fi.part = part;

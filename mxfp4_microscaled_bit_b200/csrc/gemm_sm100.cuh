@@ -278,9 +278,9 @@ struct GemmParams {
     int qhad;
     int64_t qkatoms;
     // FUSEQ: the bf16 activations [p.N rows, K] (row stride ld_xa), rotated by H_16/4 when
-    // xhad; their tensor scale is *g_w (static; the swapped form's activation slot) or, when
-    // xnpart > 0, amax / 2688 over the xnpart partial maxima at xpart, written to g_a_out by
-    // CTA 0.
+    // xhad.  Their tensor scale is *g_w (xnpart == 0: static; the swapped form's activation
+    // slot), or amax / 2688 written to g_a_out by CTA 0, the amax taken over the xnpart partial
+    // maxima at xpart (xnpart > 0) or by every CTA over all the activations (xnpart < 0).
     const __nv_bfloat16 *xa;
     int64_t ld_xa;
     int xhad;
@@ -434,6 +434,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        pdl_trigger();  // the split-K reduction may launch now; it waits for this grid to finish
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], C::FUSEQ ? 1 + C::EPI_WARPS : 1);
             mbar_init(&empty[s], 1);
@@ -590,10 +591,42 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __shared__ float s_xred[C::EPI_WARPS];
         __shared__ float s_xg;
         if constexpr (C::FUSEQ) {
-            if (p.xnpart > 0) {  // amax over the partial maxima, reduced in a fixed order
+            if (p.xnpart != 0) {  // the computed tensor scale: amax / 2688
                 float m = 0.0f;
-                for (int k = et; k < p.xnpart; k += C::EPI_WARPS * 32)
-                    m = fmaxf(m, p.xpart[k]);
+                if (p.xnpart > 0) {  // over the amax pass's partial maxima
+                    pdl_wait();  // this grid may have started before the amax pass finished
+                    for (int k = et; k < p.xnpart; k += C::EPI_WARPS * 32)
+                        m = fmaxf(m, p.xpart[k]);
+                } else {  // over all of the (few) activations, in this CTA
+                    constexpr int U = 4, T = C::EPI_WARPS * 32;
+                    const int nbk = (int)(p.K >> 4), nb = (int)p.N * nbk;
+                    for (int b0 = et; b0 < nb; b0 += U * T) {
+                        FuseRaw buf[U];
+#pragma unroll
+                        for (int j = 0; j < U; ++j) {
+                            const int b = b0 + j * T;
+                            if (b < nb) {
+                                const int r = b / nbk;
+                                const __nv_bfloat16 *src = p.xa + r * p.ld_xa + 16 * (b - r * nbk);
+                                buf[j].u0 = ld_nc_v4(src);
+                                buf[j].u1 = ld_nc_v4(src + 8);
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < U; ++j) {
+                            if (b0 + j * T < nb) {
+                                const uint32_t raw[8] = {buf[j].u0.x, buf[j].u0.y, buf[j].u0.z, buf[j].u0.w,
+                                                         buf[j].u1.x, buf[j].u1.y, buf[j].u1.z, buf[j].u1.w};
+                                float v[16];
+                                if (p.xhad)
+                                    nvfp4_block_values<true>(raw, v);
+                                else
+                                    nvfp4_block_values<false>(raw, v);
+                                m = fmaxf(m, abs_max<16>(v));
+                            }
+                        }
+                    }
+                }
 #pragma unroll
                 for (int o = 16; o; o >>= 1)
                     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -841,6 +874,7 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *ws, int
                                                             int64_t ldw, const float *g_a, const float *g_w,
                                                             __nv_bfloat16 *y, int64_t ldy, QuantOut qo)
 {
+    pdl_wait();  // launched while the GEMM still runs
     const float gg = (g_a && g_w) ? __fmul_rn(*g_a, *g_w) : 1.0f;
     const float qg = qo.qc ? *qo.qg : 1.0f;
     const int64_t nq = (N + 3) / 4, total = M * nq;

@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(QTHREADS) scale_padding_kernel(QuantShape q)
 template <bool HAD>
 __global__ void __launch_bounds__(QTHREADS) nvfp4_amax_kernel(QuantShape q, float *partials)
 {
+    pdl_trigger();  // a fused decode GEMM may start streaming its weights meanwhile
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     float m = 0.0f;
     for (int64_t seg = blockIdx.x; seg * 32 < q.blocks_per_row; seg += gridDim.x) {
