@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
                 "oracle_kv_store": (None, [u16p, i32p, ctypes.c_float, u8p, u8p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, i64, ctypes.c_int]),
                 "oracle_kv_load_fp8": (None, [u8p, u8p, i64, ctypes.c_int, ctypes.c_int, i64, ctypes.c_int, u8p]),
+                "oracle_gptq": (None, [u16p, i64, i64, i64, ctypes.c_int, ctypes.c_int, f32p, ctypes.c_float, u8p,
+                                       u8p, f32p]),
                 "oracle_kv_attention": (None, [u16p, u8p, u8p, ctypes.c_float, u8p, u8p, ctypes.c_float, i64,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, i64, ctypes.c_int, f64p]),
             }
@@ -201,6 +203,44 @@ def mxfp4_quantize(x, hadamard: int = 0, nearest: bool = False):
     fn = lib().oracle_mxfp4_quantize_nearest if nearest else lib().oracle_mxfp4_quantize
     fn(_p(xb, ctypes.c_uint16), rows, cols, cols, hadamard, _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8))
     return codes, sf
+
+
+def gptq(w, u: np.ndarray, fmt: str = "nvfp4", hadamard: int = 0, g=None, want_err: bool = False):
+    """MR-GPTQ (reading R12) of bf16 weights w [N, K] with the inverse-Hessian factor u
+    (fp32 [K, K], upper triangle read).  -> (codes [N, K/2], sf [N, K/G] row-major, g
+    (NVFP4; None for MXFP4)[, err fp32 [N, K]]).  NVFP4's g defaults to the rotated w's
+    tensor scale, as nvfp4_quantize computes it."""
+    wb = _bits(w)
+    N, K = wb.shape
+    uu = np.ascontiguousarray(u, dtype=np.float32)
+    assert uu.shape == (K, K)
+    group = 16 if fmt == "nvfp4" else 32
+    if fmt == "nvfp4" and g is None:
+        g = nvfp4_tensor_scale(wb, hadamard)
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    sf = np.zeros((N, K // group), dtype=np.uint8)
+    err = np.zeros((N, K), dtype=np.float32) if want_err else None
+    lib().oracle_gptq(_p(wb, ctypes.c_uint16), N, K, K, group, hadamard, _p(uu, ctypes.c_float),
+                      float(g) if fmt == "nvfp4" else 1.0, _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8),
+                      _p(err, ctypes.c_float) if want_err else None)
+    out = (codes, sf, np.float32(g) if fmt == "nvfp4" else None)
+    return out + (err,) if want_err else out
+
+
+def gptq_hessian_factor(x: np.ndarray, hadamard: int = 0, damp: float = 0.01) -> np.ndarray:
+    """The input GPTQ needs (reading R12), in binary64: the calibration activations x [T, K]
+    rotated blockwise by H_b / sqrt(b) (b = hadamard, 0 = none), H = x'^T x' + damp *
+    mean(diag) * I, and U upper triangular with H^-1 = U^T U; returned as float32."""
+    x = np.asarray(x, dtype=np.float64)
+    T, K = x.shape
+    if hadamard:
+        R = hadamard_matrix(hadamard).astype(np.float64) / np.sqrt(hadamard)
+        x = (x.reshape(T, K // hadamard, hadamard) @ R.T).reshape(T, K)
+    H = x.T @ x
+    H[np.diag_indices(K)] += damp * np.mean(np.diag(H))
+    Hinv = np.linalg.inv(H)
+    L = np.linalg.cholesky((Hinv + Hinv.T) / 2)
+    return np.ascontiguousarray(L.T, dtype=np.float32)
 
 
 def tc_scale_bytes(rows: int, sf_cols: int) -> int:

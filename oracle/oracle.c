@@ -54,6 +54,18 @@
  *      copy feeds attention): G query heads per kv head (query head j uses kv
  *      head j / G), scores q . k / sqrt(D) over positions 0..L-1, softmax, the
  *      p-weighted sum of the values; q bf16, output fp32; no mask beyond L.
+ *   R12 MR-GPTQ ([MRGPTQ]: GPTQ adapted to FP4 through blockwise Hadamard
+ *      transforms; [PL]: GPTQ quantises weights layer by layer with error
+ *      correction).  GPTQ's published column sweep, on the rotated weights
+ *      W' = W R (R = blockdiag(H_b / sqrt b), b = the format's block, or no
+ *      rotation) and the Hessian of the rotated inputs: U is the upper
+ *      Cholesky factor of the damped inverse Hessian (H^-1 = U^T U), an input.
+ *      Column j of every row: at the first column of each block (16 or 32) the
+ *      block's scale is fixed from the row's current values of that block by
+ *      the format's own rule (R3 with the static tensor scale g of the
+ *      rotated W, or R4); q = the dequantised code; e = (w_j - q) / U[j][j];
+ *      then w_k <- fma(-e, U[j][k], w_k) for every k > j, in binary32, so each
+ *      value receives its corrections one at a time in increasing j.
  */
 #include <math.h>
 #include <stdint.h>
@@ -384,6 +396,66 @@ EXPORT void oracle_mxfp4_quantize_nearest(const uint16_t *x, int64_t rows, int64
                                           int hadamard, uint8_t *codes, uint8_t *sf)
 {
     mxfp4_quantize_rule(x, rows, cols, ld, hadamard, codes, sf, 1);
+}
+
+/* ------------------------------------------------------------------ MR-GPTQ (R12) */
+
+/* GPTQ ([PL]: weights quantised with error correction) in the MR-GPTQ form
+ * ([MRGPTQ]: blockwise Hadamard rotations), reading R12.  GPTQ sweeps the
+ * columns in order and corrects the later columns of every row by the same
+ * rule; no step mixes two rows, so the sweep is done here one row at a time.
+ * group: 16 (NVFP4, E4M3 scales relative to g) or 32 (MXFP4, E8M0 scales).
+ * codes [N, K/2] (R6); sf [N, K/group] row-major; err [N, K] (optional): the
+ * scaled errors e, the quantities GPTQ feeds back. */
+EXPORT void oracle_gptq(const uint16_t *w, int64_t N, int64_t K, int64_t ld, int group, int hadamard,
+                        const float *u, float g, uint8_t *codes, uint8_t *sf, float *err)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t n = 0; n < N; ++n) {
+        float *row = malloc((size_t)K * sizeof(float));
+        for (int64_t b = 0; b < K / group; ++b)
+            load_block(w, ld, n, b, group, hadamard, row + b * group);
+        float d = 0.0f, rcp = 0.0f, down = 1.0f, up = 1.0f;
+        for (int64_t j = 0; j < K; ++j) {
+            if (j % group == 0) { /* the block's scale, from its current values */
+                float amax = 0.0f;
+                for (int i = 0; i < group; ++i)
+                    if (fabsf(row[j + i]) > amax)
+                        amax = fabsf(row[j + i]);
+                if (group == 16) { /* R3 */
+                    float t = (amax / 6.0f) / g;
+                    uint8_t s = oracle_e4m3_encode(t);
+                    d = (float)oracle_e4m3_decode(s) * g;
+                    rcp = (d > 0.0f) ? 1.0f / d : 0.0f;
+                    sf[n * (K / 16) + j / 16] = s;
+                } else { /* R4 */
+                    int byte = 0;
+                    if (amax > 0.0f) {
+                        int e;
+                        frexp((double)amax, &e);
+                        byte = (e - 1) - 2 + 127;
+                        if (byte < 0)
+                            byte = 0;
+                        if (byte > 254)
+                            byte = 254;
+                    }
+                    down = ldexpf(1.0f, 127 - byte);
+                    up = ldexpf(1.0f, byte - 127);
+                    sf[n * (K / 32) + j / 32] = (uint8_t)byte;
+                }
+            }
+            uint8_t c = oracle_e2m1_encode(group == 16 ? row[j] * rcp : row[j] * down);
+            float q = (float)oracle_e2m1_decode(c) * (group == 16 ? d : up);
+            uint8_t *cb = codes + n * (K / 2) + j / 2;
+            *cb = (j & 1) ? (uint8_t)(*cb | (c << 4)) : c;
+            float e = (row[j] - q) / u[j * K + j];
+            if (err)
+                err[n * K + j] = e;
+            for (int64_t k = j + 1; k < K; ++k)
+                row[k] = fmaf(-e, u[j * K + k], row[k]);
+        }
+        free(row);
+    }
 }
 
 /* ------------------------------------------------------------------ scale layout (R7) */

@@ -21,6 +21,9 @@ Workloads (the five synthetic configurations of the linear layer and the cache):
   W bf16 [14336,4096] ~ N(0, 0.02^2).  The MXFP4 comparison uses these same tensors.
 * ``kvcache`` seed 4: K and V bf16 [64,8,32768,128] ~ N(0,1) times one scale per
   (tensor, kv head), the 16 scales log-uniform on [0.1, 10].
+* ``gptq_calibration``: calibration activations for a GPTQ Hessian, float64 [T,K]:
+  Z M / sqrt(K/4) + 0.3 E with Z [T,K/4], M [K/4,K], E [T,K] ~ N(0,1) (correlated
+  channels), then K/64 channels (drawn without replacement) times 8.
 """
 from __future__ import annotations
 
@@ -31,7 +34,7 @@ import numpy as np
 import torch
 
 # tensor ids used in the generator keys
-_T_A, _T_W, _T_K, _T_V, _T_HEADSCALE, _T_OUTLIER = 1, 2, 3, 4, 5, 6
+_T_A, _T_W, _T_K, _T_V, _T_HEADSCALE, _T_OUTLIER, _T_CALIB = 1, 2, 3, 4, 5, 6, 7
 
 ROW_CHUNK = 256  # rows per independently keyed chunk
 
@@ -170,3 +173,15 @@ def normal_bf16(seed: int, rows: int, cols: int, std: float = 1.0, tag: int = 99
 
 def student_t_bf16(seed: int, rows: int, cols: int, tag: int = 98) -> torch.Tensor:
     return to_bf16(_rows(seed, tag, (rows, cols), 0, rows, cols, _student_t3))
+
+
+# ---------------------------------------------------------------- GPTQ calibration
+def gptq_calibration(seed: int, T: int, K: int) -> np.ndarray:
+    """Calibration activations [T, K] (float64): a rank-K/4 mix of normal draws plus
+    independent noise, with K/64 outlier channels times 8."""
+    g = _rng(seed, _T_CALIB, T, K)
+    z = g.standard_normal((T, K // 4))
+    m = g.standard_normal((K // 4, K)) / np.sqrt(K // 4)
+    x = z @ m + 0.3 * g.standard_normal((T, K))
+    x[:, g.choice(K, size=max(1, K // 64), replace=False)] *= 8.0
+    return x
