@@ -309,6 +309,41 @@ int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int h
                         void *y, int64_t N, int64_t ldy,
                         void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * MR-GPTQ weight quantisation (offline): GPTQ's error-correcting column sweep
+ * on the blockwise-Hadamard-rotated weights (MR-GPTQ abstract, "Abstract":
+ * GPTQ adapted to FP4 with blockwise Hadamard transforms; "FP8, NVFP4 czy
+ * AWQ?", section "Czym roznia sie FP8, NVFP4, MXFP4 i AWQ?": GPTQ quantises
+ * weights layer by layer with error correction).  For every row of
+ * W' = W blockdiag(H_b / sqrt b) (b = hadamard; 0 = no rotation), binary32:
+ * for j = 0 .. K-1: at the first column of each 16- (NVFP4) or 32-value
+ * (MXFP4) block, the block's scale is fixed from the row's current values by
+ * the format's rule (nvfp4_quantize's, relative to the tensor scale *g; or
+ * mxfp4_quantize's); q = the dequantised code of w_j; e = (w_j - q) / U[j][j];
+ * then w_k = fma(-e, U[j][k], w_k) for every k > j, in increasing j.
+ *   w: bf16 [N, K], row stride ld_w (multiple of 8), the weights as
+ *      nvfp4_quantize / mxfp4_quantize take them (unrotated);
+ *   u: float [K, K], row stride ld_u >= K: the upper Cholesky factor U of the
+ *      damped inverse Hessian of the (rotated) layer inputs, H^-1 = U^T U;
+ *      only entries with row <= column are read; U[j][j] > 0;
+ *   codes [N, K/2], scales: tensor-core layout of [N, K/16] or [N, K/32] --
+ *      ready for nvfp4_gemm / mxfp4_gemm with activations rotated the same way;
+ *   g (NVFP4): the tensor scale; compute_global_scale = 1 writes the rotated
+ *      W's amax / 2688 there (as nvfp4_quantize), 0 reads it;
+ *   workspace: gptq_workspace_bytes(N, K) bytes, 16-byte aligned (W' in
+ *      binary32 plus the block errors).
+ * K a multiple of 64.  Errors as nvfp4_quantize; a workspace below the size
+ * gives FP4LIN_ERR_WORKSPACE.  Time grows as N K^2 (binary32 multiply-adds).
+ */
+size_t gptq_workspace_bytes(int64_t N, int64_t K);
+int nvfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard,
+                        const float *u, int64_t ld_u, int compute_global_scale, float *g,
+                        uint8_t *codes, uint8_t *scales,
+                        void *workspace, size_t workspace_bytes, void *stream);
+int mxfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard,
+                        const float *u, int64_t ld_u, uint8_t *codes, uint8_t *scales,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

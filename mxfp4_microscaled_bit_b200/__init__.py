@@ -27,7 +27,8 @@ __all__ = [
     "Fp4LinError", "lib", "nvfp4_quantize", "nvfp4_gemm", "mxfp4_quantize", "mxfp4_gemm",
     "kv_nvfp4_store", "kv_nvfp4_load_fp8", "scale_bytes", "gemm_workspace_bytes",
     "device_status", "convert_selftest", "QuantizedWeight", "prepare_weight", "nvfp4_linear",
-    "mxfp4_linear", "nvfp4_linear_decode", "EXPORTS",
+    "mxfp4_linear", "nvfp4_linear_decode", "gptq_quantize", "gptq_hessian_factor", "prepare_weight_gptq",
+    "EXPORTS",
 ]
 
 STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA",
@@ -56,6 +57,9 @@ EXPORTS = {
     "nvfp4_gemm_quant": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _int, _vp, _vp, _vp, _i64, _i64, _i64,
                                 _vp, _sz, _vp]),
     "nvfp4_linear_decode_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "gptq_workspace_bytes": (_sz, [_i64, _i64]),
+    "nvfp4_gptq_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mxfp4_gptq_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_decode": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _sz,
                                    _vp]),
 }
@@ -331,6 +335,63 @@ def prepare_weight(w: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0) -> Qu
         return QuantizedWeight("nvfp4", c, s, g, hadamard, w.shape[0], w.shape[1])
     c, s = mxfp4_quantize(w, hadamard)
     return QuantizedWeight("mxfp4", c, s, None, hadamard, w.shape[0], w.shape[1])
+
+
+# ------------------------------------------------------------------ MR-GPTQ (offline weights)
+def gptq_hessian_factor(x: torch.Tensor, hadamard: int = 0, damp: float = 0.01) -> torch.Tensor:
+    """Preparation of GPTQ's input, plain dense linear algebra in float64 on x's device: the
+    calibration activations x [T, K] rotated blockwise by H_b / sqrt(b) (b = hadamard), the
+    damped Hessian H = x'^T x' + damp * mean(diag) I, and the upper factor U with
+    H^-1 = U^T U.  Returns U as float32 [K, K]."""
+    xd = x.to(torch.float64)
+    T, K = xd.shape
+    if hadamard:
+        h = torch.ones(1, 1, dtype=torch.float64, device=x.device)
+        while h.shape[0] < hadamard:
+            h = torch.cat([torch.cat([h, h], 1), torch.cat([h, -h], 1)], 0)
+        xd = (xd.reshape(T, K // hadamard, hadamard) @ (h / hadamard ** 0.5).T).reshape(T, K)
+    H = xd.T @ xd
+    H.diagonal().add_(damp * H.diagonal().mean())
+    L = torch.linalg.cholesky(H)
+    Hinv = torch.cholesky_inverse(L)
+    U = torch.linalg.cholesky((Hinv + Hinv.T) / 2, upper=True)
+    return U.to(torch.float32).contiguous()
+
+
+def gptq_quantize(w: torch.Tensor, u: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0, g=None, *,
+                  compute_global_scale: bool | None = None, codes=None, scales=None, workspace=None, stream=None):
+    """MR-GPTQ of bf16 weights w [N, K] with the inverse-Hessian factor u [K, K] (float32).
+    Returns (codes [N, K/2], scales, g) -- g None for MXFP4 -- ready for nvfp4_gemm /
+    mxfp4_gemm against activations rotated the same way."""
+    N, K = w.shape
+    dev = w.device
+    G = 16 if fmt == "nvfp4" else 32
+    if codes is None:
+        codes = torch.empty(N, K // 2, dtype=torch.uint8, device=dev)
+    if scales is None:
+        scales = torch.empty(scale_bytes(N, K // G), dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = torch.empty(int(lib().gptq_workspace_bytes(N, K)), dtype=torch.uint8, device=dev)
+    wsb = workspace.numel() * workspace.element_size()
+    if fmt == "nvfp4":
+        dynamic = (g is None) if compute_global_scale is None else bool(compute_global_scale)
+        if g is None:
+            g = torch.empty(1, dtype=torch.float32, device=dev)
+        _check("nvfp4_gptq_quantize", lib().nvfp4_gptq_quantize(
+            _ptr(w), N, K, w.stride(0), hadamard, _ptr(u), u.stride(0), int(dynamic), _ptr(g), _ptr(codes),
+            _ptr(scales), _ptr(workspace), wsb, _stream(stream)))
+        return codes, scales, g
+    _check("mxfp4_gptq_quantize", lib().mxfp4_gptq_quantize(
+        _ptr(w), N, K, w.stride(0), hadamard, _ptr(u), u.stride(0), _ptr(codes), _ptr(scales), _ptr(workspace),
+        wsb, _stream(stream)))
+    return codes, scales, None
+
+
+def prepare_weight_gptq(w: torch.Tensor, u: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0) -> "QuantizedWeight":
+    """prepare_weight with MR-GPTQ in place of plain rounding (u from gptq_hessian_factor of the
+    layer's calibration inputs with the same hadamard)."""
+    c, s, g = gptq_quantize(w, u, fmt, hadamard)
+    return QuantizedWeight(fmt, c, s, g, hadamard, w.shape[0], w.shape[1])
 
 
 def nvfp4_linear(x: torch.Tensor, w: QuantizedWeight, *, out=None, stream=None) -> torch.Tensor:

@@ -15,6 +15,7 @@
 #include "gemm_sm100_2sm.cuh"
 #include "kv.cuh"
 #include "kv_attention.cuh"
+#include "gptq.cuh"
 #include "quantize.cuh"
 #include "scale_search.cuh"
 
@@ -31,6 +32,7 @@ struct DeviceInfo {
     bool gemm_attr[7] = {false, false, false, false, false, false, false};
     int pair_clusters[2] = {0, 0};  // resident clusters of the pair kernels (0: not yet queried)
     bool attn_attr[KA_GMAX + 1] = {};  // dynamic shared memory raised for kv_attn_tc_kernel<G>
+    bool gptq_attr = false;            // dynamic shared memory raised for gptq_update_kernel
 };
 
 std::mutex g_mutex;
@@ -1025,6 +1027,131 @@ int nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld
     if (launch_status() != FP4LIN_OK)
         return FP4LIN_ERR_CUDA;
     return launch_padding(q, dev, s);
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ MR-GPTQ
+namespace {
+
+// Shared by both formats: checks, rotation, the optional tensor scale, the block sweep.
+int gptq_entry(bool nv, const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,
+               int64_t ld_u, int compute_global_scale, float *g, uint8_t *codes, uint8_t *scales, void *workspace,
+               size_t workspace_bytes, void *stream)
+{
+    const int G = nv ? 16 : 32;
+    if (!w || !u || !codes || !scales || (nv && !g) || !workspace)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (N < 1 || K < 1 || ld_w < K || ld_u < K || (hadamard != 0 && hadamard != G) ||
+        (compute_global_scale != 0 && compute_global_scale != 1))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (K % 64 != 0 || ld_w % 8 != 0 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(w, 16) || !aligned(u, 4) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(workspace, 16) ||
+        (nv && !aligned(g, 4)))
+        return FP4LIN_ERR_MISALIGNED;
+    if (workspace_bytes < gptq_workspace_bytes(N, K))
+        return FP4LIN_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (!dev->gptq_attr) {
+            if (cudaFuncSetAttribute(gptq_update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, GQ_UPD_SMEM) !=
+                cudaSuccess)
+                return FP4LIN_ERR_CUDA;
+            dev->gptq_attr = true;
+        }
+    }
+    cudaStream_t s = as_stream(stream);
+    GptqArgs a{};
+    a.wr = reinterpret_cast<float *>(workspace);
+    a.e = a.wr + N * K;
+    float *partials = a.e + N * GQ_B;
+    a.u = u;
+    a.N = N;
+    a.K = K;
+    a.ld_u = ld_u;
+    a.g = g;
+    a.codes = codes;
+    a.scales = scales;
+    a.katoms = (K / G + 3) / 4;
+    const int64_t rblocks = N * (K / G);
+    const unsigned rgrid = (unsigned)std::min<int64_t>((rblocks + 255) / 256, (int64_t)dev->sms * 16);
+    if (nv) {
+        if (hadamard)
+            gptq_rotate_kernel<16, true><<<rgrid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(w), N, K, ld_w,
+                                                               a.wr);
+        else
+            gptq_rotate_kernel<16, false><<<rgrid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(w), N, K,
+                                                                ld_w, a.wr);
+    } else {
+        if (hadamard)
+            gptq_rotate_kernel<32, true><<<rgrid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(w), N, K, ld_w,
+                                                               a.wr);
+        else
+            gptq_rotate_kernel<32, false><<<rgrid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16 *>(w), N, K,
+                                                                ld_w, a.wr);
+    }
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    if (nv && compute_global_scale) {  // g of the rotated W, as nvfp4_quantize computes it
+        QuantShape q = make_shape(w, N, K, ld_w, nullptr, nullptr, 16);
+        const dim3 agrid = amax_grid(q);
+        if (hadamard)
+            nvfp4_amax_kernel<true><<<agrid, QTHREADS, 0, s>>>(q, partials);
+        else
+            nvfp4_amax_kernel<false><<<agrid, QTHREADS, 0, s>>>(q, partials);
+        gptq_tensor_scale_kernel<<<1, 256, 0, s>>>(partials, (int)(agrid.x * agrid.y), g);
+        if (launch_status() != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+    }
+    const unsigned bgrid = (unsigned)((N + GQ_ROWS - 1) / GQ_ROWS);
+    for (int64_t c0 = 0; c0 < K; c0 += GQ_B) {
+        if (nv)
+            gptq_block_kernel<true><<<bgrid, GQ_ROWS, 0, s>>>(a, c0);
+        else
+            gptq_block_kernel<false><<<bgrid, GQ_ROWS, 0, s>>>(a, c0);
+        if (launch_status() != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+        const int64_t rest = K - c0 - GQ_B;
+        if (rest > 0) {
+            const dim3 ugrid((unsigned)((rest + GQ_TILE - 1) / GQ_TILE), (unsigned)((N + GQ_TILE - 1) / GQ_TILE));
+            gptq_update_kernel<<<ugrid, 256, GQ_UPD_SMEM, s>>>(a, c0);
+            if (launch_status() != FP4LIN_OK)
+                return FP4LIN_ERR_CUDA;
+        }
+    }
+    return launch_padding(make_shape(nullptr, N, K, K, codes, scales, G), dev, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gptq_workspace_bytes(int64_t N, int64_t K)
+{
+    if (N < 1 || K < 1)
+        return 0;
+    return (size_t)(N * K + N * GQ_B + AMAX_MAX_BLOCKS) * sizeof(float);
+}
+
+int nvfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,
+                        int64_t ld_u, int compute_global_scale, float *g, uint8_t *codes, uint8_t *scales,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    return gptq_entry(true, w, N, K, ld_w, hadamard, u, ld_u, compute_global_scale, g, codes, scales, workspace,
+                      workspace_bytes, stream);
+}
+
+int mxfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,
+                        int64_t ld_u, uint8_t *codes, uint8_t *scales, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    return gptq_entry(false, w, N, K, ld_w, hadamard, u, ld_u, 0, nullptr, codes, scales, workspace,
+                      workspace_bytes, stream);
 }
 
 }  // extern "C"

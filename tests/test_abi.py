@@ -23,7 +23,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported():
     names = header_functions()
-    assert len(names) == 20, names
+    assert len(names) == 23, names
     L = fl.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -110,6 +110,27 @@ def test_kv_argument_checks():
 
 def d(M=16, K=128, ldx=128, had=0, dyn=0, ga=P, x=P, y=P, N=64, ldy=64, ws=P, wsb=8192):
     return fl.lib().nvfp4_linear_decode(x, M, K, ldx, had, dyn, ga, P, P, P, y, N, ldy, ws, wsb, None)
+
+
+def test_gptq_argument_checks():
+    L = fl.lib()
+    ws = L.gptq_workspace_bytes(64, 128)
+    assert ws == (64 * 128 + 64 * 64 + 1024) * 4
+
+    def q(w=P, N=64, K=128, ldw=128, had=0, u=P, ldu=128, dyn=0, g=P, wsp=P, wsb=ws):
+        return L.nvfp4_gptq_quantize(w, N, K, ldw, had, u, ldu, dyn, g, P, P, wsp, wsb, None)
+
+    assert q(w=None) == INVALID
+    assert q(u=None) == INVALID
+    assert q(g=None) == INVALID
+    assert q(had=32) == INVALID
+    assert q(ldu=64) == INVALID
+    assert q(K=96, ldw=96, ldu=96) == SHAPE
+    assert q(u=P + 2) == MISALIGNED
+    assert q(wsb=ws - 1) == WORKSPACE
+    assert q(wsp=None) == INVALID
+    assert L.mxfp4_gptq_quantize(P, 64, 128, 128, 16, P, 128, P, P, P, ws, None) == INVALID  # 32 or 0
+    assert L.mxfp4_gptq_quantize(P, 64, 96, 96, 32, P, 96, P, P, P, ws, None) == SHAPE
 
 
 def test_linear_decode_argument_checks():
