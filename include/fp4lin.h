@@ -323,15 +323,20 @@ int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int h
  * then w_k = fma(-e, U[j][k], w_k) for every k > j, in increasing j.
  *   w: bf16 [N, K], row stride ld_w (multiple of 8), the weights as
  *      nvfp4_quantize / mxfp4_quantize take them (unrotated);
- *   u: float [K, K], row stride ld_u >= K: the upper Cholesky factor U of the
- *      damped inverse Hessian of the (rotated) layer inputs, H^-1 = U^T U;
- *      only entries with row <= column are read; U[j][j] > 0;
+ *   u: float [K, K], row stride ld_u >= K (a multiple of 4; u 16-byte
+ *      aligned): the upper Cholesky factor U of the damped inverse Hessian of
+ *      the (rotated) layer inputs, H^-1 = U^T U; only entries with row <=
+ *      column are read; U[j][j] > 0;
  *   codes [N, K/2], scales: tensor-core layout of [N, K/16] or [N, K/32] --
  *      ready for nvfp4_gemm / mxfp4_gemm with activations rotated the same way;
  *   g (NVFP4): the tensor scale; compute_global_scale = 1 writes the rotated
  *      W's amax / 2688 there (as nvfp4_quantize), 0 reads it;
  *   workspace: gptq_workspace_bytes(N, K) bytes, 16-byte aligned (W' in
- *      binary32 plus the block errors).
+ *      binary32, the errors of two 256-column superblocks, the tensor-scale
+ *      partials).
+ * The work forks from `stream` onto two streams the call creates (the column
+ * sweep at the highest priority, the bulk corrections at the lowest) and joins
+ * back into it before the call returns; both are released with the call.
  * K a multiple of 64.  Errors as nvfp4_quantize; a workspace below the size
  * gives FP4LIN_ERR_WORKSPACE.  Time grows as N K^2 (binary32 multiply-adds).
  */

@@ -1034,6 +1034,59 @@ int nvfp4_quantize_noalloc(const void *x, int64_t rows, int64_t cols, int64_t ld
 // ------------------------------------------------------------------ MR-GPTQ
 namespace {
 
+// The two internal streams of one GPTQ call and the events that order them; everything is
+// released when the call returns (CUDA frees a stream or event once its pending work is done).
+struct GptqStreams {
+    cudaStream_t user = nullptr, chain = nullptr, bulk = nullptr;
+    cudaEvent_t ev[64];
+    int nev = 0;
+    bool joined = false;
+
+    bool record_wait(cudaStream_t from, cudaStream_t to)  // `to` waits for the work queued on `from`
+    {
+        if (nev == 64) {  // reuse: a recorded event may be re-recorded once the wait is queued
+            for (int i = 0; i < nev; ++i)
+                cudaEventDestroy(ev[i]);
+            nev = 0;
+        }
+        cudaEvent_t e;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+            return false;
+        ev[nev++] = e;
+        return cudaEventRecord(e, from) == cudaSuccess && cudaStreamWaitEvent(to, e, 0) == cudaSuccess;
+    }
+    bool fork(cudaStream_t u)
+    {
+        user = u;
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&chain, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&bulk, cudaStreamNonBlocking, least) != cudaSuccess)
+            return false;
+        return record_wait(user, chain) && record_wait(user, bulk);
+    }
+    bool order(cudaStream_t first, cudaStream_t then) { return record_wait(first, then); }
+    bool join()
+    {
+        joined = record_wait(chain, user) && record_wait(bulk, user);
+        return joined;
+    }
+    ~GptqStreams()
+    {
+        if (!joined && user && chain && bulk) {  // an error path: still leave nothing dangling in the caller's stream
+            record_wait(chain, user);
+            record_wait(bulk, user);
+        }
+        for (int i = 0; i < nev; ++i)
+            cudaEventDestroy(ev[i]);
+        if (chain)
+            cudaStreamDestroy(chain);
+        if (bulk)
+            cudaStreamDestroy(bulk);
+        cudaGetLastError();
+    }
+};
+
 // Shared by both formats: checks, rotation, the optional tensor scale, the block sweep.
 int gptq_entry(bool nv, const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,
                int64_t ld_u, int compute_global_scale, float *g, uint8_t *codes, uint8_t *scales, void *workspace,
@@ -1045,9 +1098,9 @@ int gptq_entry(bool nv, const void *w, int64_t N, int64_t K, int64_t ld_w, int h
     if (N < 1 || K < 1 || ld_w < K || ld_u < K || (hadamard != 0 && hadamard != G) ||
         (compute_global_scale != 0 && compute_global_scale != 1))
         return FP4LIN_ERR_INVALID_ARGUMENT;
-    if (K % 64 != 0 || ld_w % 8 != 0 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+    if (K % 64 != 0 || ld_w % 8 != 0 || ld_u % 4 != 0 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
         return FP4LIN_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned(w, 16) || !aligned(u, 4) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(workspace, 16) ||
+    if (!aligned(w, 16) || !aligned(u, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(workspace, 16) ||
         (nv && !aligned(g, 4)))
         return FP4LIN_ERR_MISALIGNED;
     if (workspace_bytes < gptq_workspace_bytes(N, K))
@@ -1065,11 +1118,20 @@ int gptq_entry(bool nv, const void *w, int64_t N, int64_t K, int64_t ld_w, int h
             dev->gptq_attr = true;
         }
     }
-    cudaStream_t s = as_stream(stream);
+    // Two streams forked from (and joined back into) the caller's: the sweep chain at the
+    // highest priority, the bulk trailing corrections at the lowest, so that the latency-bound
+    // sweep of superblock s+1 runs while the corrections of superblock s stream into the rest
+    // of W'.  The two touch disjoint columns, and E^T alternates between two buffers.
+    GptqStreams gs;
+    if (!gs.fork(as_stream(stream)))
+        return FP4LIN_ERR_CUDA;
+    cudaStream_t s = gs.chain, bs = gs.bulk;
     GptqArgs a{};
     a.wr = reinterpret_cast<float *>(workspace);
-    a.e = a.wr + N * K;
-    float *partials = a.e + N * GQ_B;
+    a.np = (N + 3) / 4 * 4;
+    float *et_base = a.wr + N * K;
+    float *partials = et_base + 2 * GQ_SB * a.np;
+    a.et = et_base;
     a.u = u;
     a.N = N;
     a.K = K;
@@ -1109,22 +1171,44 @@ int gptq_entry(bool nv, const void *w, int64_t N, int64_t K, int64_t ld_w, int h
             return FP4LIN_ERR_CUDA;
     }
     const unsigned bgrid = (unsigned)((N + GQ_ROWS - 1) / GQ_ROWS);
-    for (int64_t c0 = 0; c0 < K; c0 += GQ_B) {
-        if (nv)
-            gptq_block_kernel<true><<<bgrid, GQ_ROWS, 0, s>>>(a, c0);
-        else
-            gptq_block_kernel<false><<<bgrid, GQ_ROWS, 0, s>>>(a, c0);
-        if (launch_status() != FP4LIN_OK)
-            return FP4LIN_ERR_CUDA;
-        const int64_t rest = K - c0 - GQ_B;
-        if (rest > 0) {
-            const dim3 ugrid((unsigned)((rest + GQ_TILE - 1) / GQ_TILE), (unsigned)((N + GQ_TILE - 1) / GQ_TILE));
-            gptq_update_kernel<<<ugrid, 256, GQ_UPD_SMEM, s>>>(a, c0);
+    const unsigned rtiles = (unsigned)((N + GQ_TILE - 1) / GQ_TILE);
+    // corrections of columns j0 .. j0+nj-1 (E^T rows jo ..) to the columns [k0, k1)
+    auto update = [&](cudaStream_t st, int64_t j0, int nj, int64_t jo, int64_t k0, int64_t k1) {
+        const dim3 ugrid((unsigned)((k1 - k0 + GQ_TILE - 1) / GQ_TILE), rtiles);
+        gptq_update_kernel<<<ugrid, 256, GQ_UPD_SMEM, st>>>(a, j0, nj, jo, k0, k1);
+        return launch_status();
+    };
+    bool bulk_pending = false;
+    for (int64_t s0 = 0; s0 < K; s0 += GQ_SB) {
+        const int64_t s1 = std::min<int64_t>(K, s0 + GQ_SB), s2 = std::min<int64_t>(K, s1 + GQ_SB);
+        a.et = et_base + ((s0 / GQ_SB) & 1) * GQ_SB * a.np;
+        for (int64_t c0 = s0; c0 < s1; c0 += GQ_B) {
+            if (nv)
+                gptq_block_kernel<true><<<bgrid, GQ_ROWS, 0, s>>>(a, c0, s0);
+            else
+                gptq_block_kernel<false><<<bgrid, GQ_ROWS, 0, s>>>(a, c0, s0);
             if (launch_status() != FP4LIN_OK)
                 return FP4LIN_ERR_CUDA;
+            if (c0 + GQ_B < s1 && update(s, c0, GQ_B, c0 - s0, c0 + GQ_B, s1) != FP4LIN_OK)  // rest of the superblock
+                return FP4LIN_ERR_CUDA;
+        }
+        if (s1 == K)
+            break;
+        // the next superblock's columns: after the previous superblock's bulk corrections
+        if (bulk_pending && !gs.order(bs, s))
+            return FP4LIN_ERR_CUDA;
+        if (update(s, s0, (int)(s1 - s0), 0, s1, s2) != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+        // everything after it, on the bulk stream, once this superblock's errors are written
+        if (s2 < K) {
+            if (!gs.order(s, bs) || update(bs, s0, (int)(s1 - s0), 0, s2, K) != FP4LIN_OK)
+                return FP4LIN_ERR_CUDA;
+            bulk_pending = true;
         }
     }
-    return launch_padding(make_shape(nullptr, N, K, K, codes, scales, G), dev, s);
+    if (launch_padding(make_shape(nullptr, N, K, K, codes, scales, G), dev, s) != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    return gs.join() ? FP4LIN_OK : FP4LIN_ERR_CUDA;
 }
 
 }  // namespace
@@ -1135,7 +1219,7 @@ size_t gptq_workspace_bytes(int64_t N, int64_t K)
 {
     if (N < 1 || K < 1)
         return 0;
-    return (size_t)(N * K + N * GQ_B + AMAX_MAX_BLOCKS) * sizeof(float);
+    return (size_t)(N * K + 2 * GQ_SB * ((N + 3) / 4 * 4) + AMAX_MAX_BLOCKS) * sizeof(float);
 }
 
 int nvfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,

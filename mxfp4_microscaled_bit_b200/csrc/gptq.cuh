@@ -11,15 +11,20 @@
 // U (upper triangular, H^-1 = U^T U for the damped Hessian of the rotated inputs) is an
 // input.
 //
-// GPU form (GPTQ's lazy batches, in the same arithmetic order):
+// GPU form (GPTQ's lazy batches, two levels deep, in the same arithmetic order):
 //  * gptq_rotate_kernel: bf16 W -> binary32 W' in the workspace (the quantisers' rotation).
-//  * per 64-column block [c0, c0+64):
+//  * per superblock of 256 columns [s0, s0+256), per 64-column block [c0, c0+64) in it:
 //      gptq_block_kernel: one thread per row holds the 64 values in registers and sweeps
 //      them, reading the 64x64 triangle of U from shared memory (every thread reads the same
-//      word: a broadcast); writes the codes, the scales and the 64 errors e of its row;
-//      gptq_update_kernel: W'[:, c0+64:] receives the block's corrections, element by
-//      element in increasing j -- a 128x128-tile binary32 product accumulated straight into
-//      W', with E and U staged in shared memory.
+//      word: a broadcast); writes the codes, the scales and the negated errors -e of its
+//      row into E^T [256][N] (transposed: the update kernel copies it as it stands);
+//      gptq_update_kernel over [c0+64, s0+256): the block's corrections to the rest of the
+//      superblock, so the next block sweeps current values;
+//    then gptq_update_kernel over [s0+256, K) with all 256 corrections of the superblock.
+//    Each value still receives its corrections one at a time in increasing j; W' beyond the
+//    superblock is read and written once per 256 columns instead of once per 64.
+//  The update is a 128x128-tile binary32 product accumulated straight into W', its E and U
+//  chunks streamed through a double-buffered cp.async ring.
 // The tensor cores are not used: their products round differently, and the quantisation
 // decisions downstream must see exactly the binary32 values the sweep defines.
 #pragma once
@@ -29,14 +34,17 @@
 namespace fp4lin {
 
 constexpr int GQ_B = 64;         // columns per lazy block
+constexpr int GQ_SB = 256;       // columns per superblock (the E^T buffer's height)
 constexpr int GQ_ROWS = 128;     // rows (threads) per CTA of the block kernel
 constexpr int GQ_TILE = 128;     // update kernel: 128 x 128 tile of W', 256 threads, 8 x 8 each
-constexpr int GQ_ES = GQ_TILE + 1;  // padded row of the transposed E tile (conflict-free stores)
-constexpr int GQ_UPD_SMEM = (GQ_B * GQ_ES + GQ_B * GQ_TILE) * 4;
+constexpr int GQ_CJ = 32;                                        // values of j per staged chunk
+constexpr int GQ_CHUNK_FLOATS = GQ_CJ * GQ_TILE;                 // one 32 x 128 operand chunk
+constexpr int GQ_UPD_SMEM = 2 * 2 * GQ_CHUNK_FLOATS * 4;          // two stages of (E^T chunk, U chunk): 64 KB
 
 struct GptqArgs {
     float *wr;            // W' [N, K] binary32, row stride K (workspace)
-    float *e;             // errors of the current block [N, 64] (workspace)
+    float *et;            // -e of the current superblock, transposed: [256][np] (workspace)
+    int64_t np;           // row stride of et: N rounded up to a multiple of 4
     const float *u;       // U [K, K], row stride ld_u; entries with row > column are not read
     int64_t N, K, ld_u;
     const float *g;       // NVFP4 tensor scale (device)
@@ -119,7 +127,7 @@ template <bool NV, int J>
 struct GptqColumn {
     static __device__ __forceinline__ void run(float (&w)[GQ_B], const float (&us)[GQ_B][GQ_B], float g, float &mul,
                                                float &back, uint32_t (&code_words)[GQ_B / 8], uint32_t &sf_word,
-                                               float *erow)
+                                               float *ecol, int64_t np)
     {
         constexpr int G = NV ? 16 : 32;
         if constexpr (J % G == 0) {
@@ -146,19 +154,19 @@ struct GptqColumn {
         else
             code_words[J / 8] |= c << (4 * (J % 8));
         const float e = __fdiv_rn(__fsub_rn(w[J], q), us[J][J]);
-        erow[J] = e;
+        ecol[J * np] = -e;
 #pragma unroll
         for (int k = J + 1; k < GQ_B; ++k)
             w[k] = __fmaf_rn(-e, us[J][k], w[k]);
         if constexpr (J + 1 < GQ_B)
-            GptqColumn<NV, J + 1>::run(w, us, g, mul, back, code_words, sf_word, erow);
+            GptqColumn<NV, J + 1>::run(w, us, g, mul, back, code_words, sf_word, ecol, np);
     }
 };
 
 // One 64-column block of the sweep for every row.  NV: NVFP4 (16-value blocks, E4M3 scales
 // relative to *g); else MXFP4 (32-value blocks, E8M0 scales by the OCP exponent rule).
 template <bool NV>
-__global__ void __launch_bounds__(GQ_ROWS) gptq_block_kernel(GptqArgs a, int64_t c0)
+__global__ void __launch_bounds__(GQ_ROWS) gptq_block_kernel(GptqArgs a, int64_t c0, int64_t s0)
 {
     __shared__ float us[GQ_B][GQ_B];
     for (int i = threadIdx.x; i < GQ_B * GQ_B; i += GQ_ROWS) {
@@ -183,7 +191,7 @@ __global__ void __launch_bounds__(GQ_ROWS) gptq_block_kernel(GptqArgs a, int64_t
     float mul = 0.0f, back = 0.0f;  // x -> code scale and code -> value scale of the current block
     uint32_t code_words[GQ_B / 8];
     uint32_t sf_word = 0;
-    GptqColumn<NV, 0>::run(w, us, g, mul, back, code_words, sf_word, a.e + n * GQ_B);
+    GptqColumn<NV, 0>::run(w, us, g, mul, back, code_words, sf_word, a.et + (c0 - s0) * a.np + n, a.np);
     uint4 *dst = reinterpret_cast<uint4 *>(a.codes + n * (a.K / 2) + c0 / 2);
     dst[0] = make_uint4(code_words[0], code_words[1], code_words[2], code_words[3]);
     dst[1] = make_uint4(code_words[4], code_words[5], code_words[6], code_words[7]);
@@ -193,34 +201,55 @@ __global__ void __launch_bounds__(GQ_ROWS) gptq_block_kernel(GptqArgs a, int64_t
         *reinterpret_cast<uint16_t *>(a.scales + tc_offset(n, c0 / 32, a.katoms)) = (uint16_t)sf_word;
 }
 
-// W'[:, c0+64 : K] -= (the block's corrections), element by element in increasing j:
-// w = fma(-e_j, U[c0+j][k], w) for j = 0..63.  CTA tile 128 rows x 128 columns; thread
-// (ty, tx) of 16 x 16 holds rows ty + 16 i (i < 8) and columns 4 tx + 64 h + l (h < 2, l < 4).
-__global__ void __launch_bounds__(256) gptq_update_kernel(GptqArgs a, int64_t c0)
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, uint32_t src_bytes)
 {
-    extern __shared__ float gq_smem[];
-    float *es = gq_smem;                  // [64][GQ_ES]: es[j][r] = e[row0 + r][j]
-    float *us = gq_smem + GQ_B * GQ_ES;   // [64][128]:   us[j][c] = U[c0 + j][col0 + c]
-    const int64_t c1 = c0 + GQ_B;
-    const int64_t row0 = (int64_t)blockIdx.y * GQ_TILE, col0 = c1 + (int64_t)blockIdx.x * GQ_TILE;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// W'[:, k0 : k1) receives the corrections of columns j0 .. j0+nj-1 (nj a multiple of 64),
+// element by element in increasing j: w = fma(-e_j, U[j][k], w).  -e_j comes from row
+// jo + (j - j0) of E^T.  CTA tile 128 rows x 128 columns; thread (ty, tx) of 16 x 16 holds
+// rows 8 ty + i (i < 8) and columns 4 tx + 64 h + l (h < 2, l < 4), so a step j is four
+// 128-bit shared loads (8 multipliers, 8 U values) and 64 scalar fmas.  (The packed
+// fma.rn.f32x2 form holds the FMA pipe two cycles per instruction and measured slower.)
+__global__ void __launch_bounds__(256, 2)
+    gptq_update_kernel(GptqArgs a, int64_t j0, int nj, int64_t jo, int64_t k0, int64_t k1)
+{
+    extern __shared__ __align__(16) float gq_smem[];
+    const int64_t row0 = (int64_t)blockIdx.y * GQ_TILE, col0 = k0 + (int64_t)blockIdx.x * GQ_TILE;
     const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
-    for (int i = t; i < GQ_B * GQ_TILE; i += 256) {
-        const int r = i / GQ_B, j = i % GQ_B;  // consecutive threads: consecutive j of one row
-        const int64_t n = row0 + r;
-        es[j * GQ_ES + r] = n < a.N ? a.e[n * GQ_B + j] : 0.0f;
-        const int jj = i / GQ_TILE, c = i % GQ_TILE;
-        const int64_t k = col0 + c;
-        us[jj * GQ_TILE + c] = k < a.K ? a.u[(c0 + jj) * a.ld_u + k] : 0.0f;
-    }
+    // chunk q (32 values of j) into stage b: es[j][r] = -e of row row0 + r, us[j][c] = U[j][col0 + c]
+    auto stage = [&](int q, int b) {
+        float *es = gq_smem + b * 2 * GQ_CHUNK_FLOATS, *us = es + GQ_CHUNK_FLOATS;
+#pragma unroll
+        for (int x = 0; x < GQ_CHUNK_FLOATS / 4 / 256; ++x) {
+            const int c = t + 256 * x, j = c >> 5, q4 = (c & 31) * 4;  // 32 16-byte pieces per row
+            const int64_t n = row0 + q4;
+            const int64_t nv = a.N - n;  // rows of this piece inside E^T's live part
+            const uint32_t eb = nv >= 4 ? 16u : nv > 0 ? (uint32_t)nv * 4u : 0u;
+            const float *esrc = a.et + (jo + GQ_CJ * q + j) * a.np + (eb ? n : 0);
+            cp_async16(es + j * GQ_TILE + q4, esrc, eb);
+            const int64_t k = col0 + q4;
+            const uint32_t ub = k < k1 ? 16u : 0u;  // k1 - col0 is a multiple of 64: whole pieces
+            const float *usrc = a.u + (j0 + GQ_CJ * q + j) * a.ld_u + (ub ? k : 0);
+            cp_async16(us + j * GQ_TILE + q4, usrc, ub);
+        }
+    };
+    const int nq = nj / GQ_CJ;
+    stage(0, 0);
+    cp_async_commit();
     float acc[8][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int64_t n = row0 + ty + 16 * i;
+        const int64_t n = row0 + 8 * ty + i;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            const int64_t k = col0 + 4 * tx + 64 * h;  // K - c1 is a multiple of 64: 4 columns all in or all out
+            const int64_t k = col0 + 4 * tx + 64 * h;
             float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (n < a.N && k < a.K)
+            if (n < a.N && k < k1)
                 v = *reinterpret_cast<const float4 *>(a.wr + n * a.K + k);
             acc[i][4 * h] = v.x;
             acc[i][4 * h + 1] = v.y;
@@ -228,30 +257,36 @@ __global__ void __launch_bounds__(256) gptq_update_kernel(GptqArgs a, int64_t c0
             acc[i][4 * h + 3] = v.w;
         }
     }
-    __syncthreads();
-#pragma unroll 4
-    for (int j = 0; j < GQ_B; ++j) {
-        float ev[8], uv[8];
+    for (int q = 0; q < nq; ++q) {
+        if (q + 1 < nq)
+            stage(q + 1, (q + 1) & 1);
+        cp_async_commit();  // possibly empty: the wait below always leaves one group in flight
+        cp_async_wait1();
+        __syncthreads();
+        const float *es = gq_smem + (q & 1) * 2 * GQ_CHUNK_FLOATS, *us = es + GQ_CHUNK_FLOATS;
+#pragma unroll 2
+        for (int j = 0; j < GQ_CJ; ++j) {
+            const float4 e0 = *reinterpret_cast<const float4 *>(es + j * GQ_TILE + 8 * ty);
+            const float4 e1 = *reinterpret_cast<const float4 *>(es + j * GQ_TILE + 8 * ty + 4);
+            const float4 u0 = *reinterpret_cast<const float4 *>(us + j * GQ_TILE + 4 * tx);
+            const float4 u1 = *reinterpret_cast<const float4 *>(us + j * GQ_TILE + 64 + 4 * tx);
+            const float ev[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+            const float uv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            ev[i] = -es[j * GQ_ES + ty + 16 * i];
-        const float4 u0 = *reinterpret_cast<const float4 *>(us + j * GQ_TILE + 4 * tx);
-        const float4 u1 = *reinterpret_cast<const float4 *>(us + j * GQ_TILE + 64 + 4 * tx);
-        uv[0] = u0.x; uv[1] = u0.y; uv[2] = u0.z; uv[3] = u0.w;
-        uv[4] = u1.x; uv[5] = u1.y; uv[6] = u1.z; uv[7] = u1.w;
+            for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int l = 0; l < 8; ++l)
-                acc[i][l] = __fmaf_rn(ev[i], uv[l], acc[i][l]);
+                for (int l = 0; l < 8; ++l)
+                    acc[i][l] = __fmaf_rn(ev[i], uv[l], acc[i][l]);
+        }
+        __syncthreads();  // stage q & 1 is refilled by the next iteration
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const int64_t n = row0 + ty + 16 * i;
+        const int64_t n = row0 + 8 * ty + i;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int64_t k = col0 + 4 * tx + 64 * h;
-            if (n < a.N && k < a.K)
+            if (n < a.N && k < k1)
                 *reinterpret_cast<float4 *>(a.wr + n * a.K + k) =
                     make_float4(acc[i][4 * h], acc[i][4 * h + 1], acc[i][4 * h + 2], acc[i][4 * h + 3]);
         }

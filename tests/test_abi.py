@@ -115,7 +115,7 @@ def d(M=16, K=128, ldx=128, had=0, dyn=0, ga=P, x=P, y=P, N=64, ldy=64, ws=P, ws
 def test_gptq_argument_checks():
     L = fl.lib()
     ws = L.gptq_workspace_bytes(64, 128)
-    assert ws == (64 * 128 + 64 * 64 + 1024) * 4
+    assert ws == (64 * 128 + 2 * 256 * 64 + 1024) * 4
 
     def q(w=P, N=64, K=128, ldw=128, had=0, u=P, ldu=128, dyn=0, g=P, wsp=P, wsb=ws):
         return L.nvfp4_gptq_quantize(w, N, K, ldw, had, u, ldu, dyn, g, P, P, wsp, wsb, None)
@@ -126,7 +126,8 @@ def test_gptq_argument_checks():
     assert q(had=32) == INVALID
     assert q(ldu=64) == INVALID
     assert q(K=96, ldw=96, ldu=96) == SHAPE
-    assert q(u=P + 2) == MISALIGNED
+    assert q(u=P + 4) == MISALIGNED
+    assert q(ldu=130) == SHAPE
     assert q(wsb=ws - 1) == WORKSPACE
     assert q(wsp=None) == INVALID
     assert L.mxfp4_gptq_quantize(P, 64, 128, 128, 16, P, 128, P, P, P, ws, None) == INVALID  # 32 or 0
