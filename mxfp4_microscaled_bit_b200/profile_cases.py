@@ -7,7 +7,9 @@ cases: gemm_prefill (8192 x 14336 x 4096 NVFP4, 16-wide rotation), gemm_mxfp4,
 gemm_decode (16 x 14336 x 4096), quant_prefill (8192 x 4096 rotated, dynamic
 scale), kv_load (8 x 8 x 32768 x 128 cache to FP8), kv_store, kv_attention (decode
 attention over the same 8 x 8 caches, G = 4), quant_mse (the 14336 x 4096 weight,
-MSE-optimal scales), gemm_quant (the prefill GEMM with its output NVFP4-encoded).
+MSE-optimal scales), gemm_quant (the prefill GEMM with its output NVFP4-encoded),
+linear_decode (16 x 14336 x 4096 with the activation quantiser inside the GEMM),
+gptq (MR-GPTQ of the 14336 x 4096 weight, NVFP4, 16-wide rotation).
 """
 from __future__ import annotations
 
@@ -28,12 +30,27 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
                     choices=["gemm_prefill", "gemm_mxfp4", "gemm_decode", "quant_prefill", "kv_load", "kv_store",
-                             "kv_attention", "quant_mse", "gemm_quant"])
+                             "kv_attention", "quant_mse", "gemm_quant", "linear_decode", "gptq"])
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    if a.case == "quant_mse":
+    if a.case == "gptq":
+        W = si.prefill_W().to(dev)
+        K = W.shape[1]
+        u = fl.gptq_hessian_factor(torch.from_numpy(si.gptq_calibration(7, 2 * K, K)).to(dev), 16)
+        ws = torch.empty(int(fl.lib().gptq_workspace_bytes(W.shape[0], K)), dtype=torch.uint8, device=dev)
+        fn = lambda: fl.gptq_quantize(W, u, "nvfp4", 16, workspace=ws)  # noqa: E731
+    elif a.case == "linear_decode":
+        M, N, K = 16, 14336, 4096
+        w = fl.prepare_weight(si.decode_W(N, K).to(dev), "nvfp4", 0)
+        x = si.decode_A(M, K).to(dev)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        g = torch.empty(1, dtype=torch.float32, device=dev)
+        ws = torch.empty(int(fl.lib().nvfp4_linear_decode_workspace_bytes(M, N, K)), dtype=torch.uint8, device=dev)
+        fn = lambda: fl.nvfp4_linear_decode(x, w.codes, w.scales, w.g, g_a=g, compute_global_scale=True,  # noqa: E731
+                                            out=y, workspace=ws)
+    elif a.case == "quant_mse":
         W = si.prefill_W().to(dev)
         fn = lambda: fl.nvfp4_quantize(W, 16, mse=True)  # noqa: E731
     elif a.case in ("gemm_prefill", "gemm_mxfp4", "quant_prefill", "gemm_quant"):
