@@ -349,6 +349,34 @@ int mxfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int h
                         const float *u, int64_t ld_u, uint8_t *codes, uint8_t *scales,
                         void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Decode weights in tile order.  The decode-sized GEMM (M <= 16) streams the
+ * weights 128 rows x 256 values at a time.  In the row-major layout each such
+ * stage is 128 strided runs of 128 bytes; prepared once in tile order, each
+ * stage is one contiguous 16 KB block that a bulk copy lands in shared memory
+ * as the exact 128-byte-swizzled operand image (16-byte chunk c of row r at
+ * position c ^ (r % 8)).  Tile (mt, kt) -- rows 128 mt .. +127, code bytes
+ * 128 kt .. +127 -- starts at byte (mt * ceil(K/256) + kt) * 16384; rows past N
+ * and bytes past K/2 are zero.  The scales stay in the tensor-core layout.
+ *   fp4lin_tiled_weight_bytes(N, K): the tiled buffer's size.
+ *   fp4lin_tile_weights: codes [N, K/2] (as nvfp4_quantize writes them) -> tiled.
+ *   nvfp4_gemm_tiled, nvfp4_linear_decode_tiled: nvfp4_gemm / nvfp4_linear_decode
+ *   with the weights' codes in tile order (w_tiled); same results, bit for bit;
+ *   M <= 16 (else FP4LIN_ERR_UNSUPPORTED_SHAPE).  K a multiple of 64; pointers
+ *   16-byte aligned.  Errors as the untiled calls.
+ */
+size_t fp4lin_tiled_weight_bytes(int64_t N, int64_t K);
+int fp4lin_tile_weights(const uint8_t *codes, int64_t N, int64_t K, uint8_t *tiled, void *stream);
+int nvfp4_gemm_tiled(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a,
+                     const uint8_t *w_tiled, const uint8_t *w_scales, const float *g_w,
+                     void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+                     void *workspace, size_t workspace_bytes, void *stream);
+int nvfp4_linear_decode_tiled(const void *x, int64_t M, int64_t K, int64_t ld_x, int hadamard,
+                              int compute_global_scale, float *g_a,
+                              const uint8_t *w_tiled, const uint8_t *w_scales, const float *g_w,
+                              void *y, int64_t N, int64_t ldy,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

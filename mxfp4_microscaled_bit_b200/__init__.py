@@ -27,7 +27,7 @@ __all__ = [
     "Fp4LinError", "lib", "nvfp4_quantize", "nvfp4_gemm", "mxfp4_quantize", "mxfp4_gemm",
     "kv_nvfp4_store", "kv_nvfp4_load_fp8", "scale_bytes", "gemm_workspace_bytes",
     "device_status", "convert_selftest", "QuantizedWeight", "prepare_weight", "nvfp4_linear",
-    "mxfp4_linear", "nvfp4_linear_decode", "gptq_quantize", "gptq_hessian_factor", "prepare_weight_gptq",
+    "mxfp4_linear", "nvfp4_linear_decode", "tile_weights", "nvfp4_gemm_tiled", "gptq_quantize", "gptq_hessian_factor", "prepare_weight_gptq",
     "EXPORTS",
 ]
 
@@ -58,6 +58,11 @@ EXPORTS = {
                                 _vp, _sz, _vp]),
     "nvfp4_linear_decode_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "gptq_workspace_bytes": (_sz, [_i64, _i64]),
+    "fp4lin_tiled_weight_bytes": (_sz, [_i64, _i64]),
+    "fp4lin_tile_weights": (_int, [_vp, _i64, _i64, _vp, _vp]),
+    "nvfp4_gemm_tiled": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp]),
+    "nvfp4_linear_decode_tiled": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
+                                         _vp, _sz, _vp]),
     "nvfp4_gptq_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_gptq_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_decode": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _sz,
@@ -245,14 +250,36 @@ def nvfp4_gemm_quant(a_codes, a_scales, g_a, w_codes, w_scales, g_w, g_y, *, had
     return y, y_codes, y_scales
 
 
+def tile_weights(codes: torch.Tensor, *, stream=None) -> torch.Tensor:
+    """Weight codes [N, K/2] -> the decode GEMM's tile order (flat uint8, see include/fp4lin.h)."""
+    N, K = codes.shape[0], codes.shape[1] * 2
+    tiled = torch.empty(int(lib().fp4lin_tiled_weight_bytes(N, K)), dtype=torch.uint8, device=codes.device)
+    _check("fp4lin_tile_weights", lib().fp4lin_tile_weights(_ptr(codes), N, K, _ptr(tiled), _stream(stream)))
+    return tiled
+
+
+def nvfp4_gemm_tiled(a_codes, a_scales, g_a, w_tiled, w_scales, g_w, N: int, *, out=None, workspace=None,
+                     stream=None):
+    """nvfp4_gemm for M <= 16 with the weights' codes in tile order (tile_weights)."""
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    y = _gemm_out(M, N, out, a_codes.device)
+    ws, wsb = _gemm_ws(M, N, K, workspace, a_codes.device)
+    _check("nvfp4_gemm_tiled", lib().nvfp4_gemm_tiled(
+        _ptr(a_codes), _ptr(a_scales), _ptr(g_a), _ptr(w_tiled), _ptr(w_scales), _ptr(g_w), _ptr(y), M, N, K,
+        y.stride(0), _ptr(ws), wsb, _stream(stream)))
+    return y
+
+
 def nvfp4_linear_decode(x, w_codes, w_scales, g_w, *, hadamard: int = 0, g_a=None,
-                        compute_global_scale: bool | None = None, out=None, workspace=None, stream=None):
+                        compute_global_scale: bool | None = None, out=None, workspace=None, stream=None,
+                        tiled_n: int | None = None):
     """Decode-sized (M <= 16) y = x W^T with the activation quantiser inside the GEMM: bit-equal to
     nvfp4_quantize(x, hadamard, g_a, compute_global_scale=...) then nvfp4_gemm.  The activations'
     tensor scale is computed (amax / 2688) when g_a is None or compute_global_scale is True (then
-    written into g_a), else taken from g_a.  Returns (y, g_a)."""
+    written into g_a), else taken from g_a.  tiled_n: w_codes is the tile-order buffer of a
+    weight with tiled_n rows (tile_weights).  Returns (y, g_a)."""
     M, K = x.shape
-    N = w_codes.shape[0]
+    N = w_codes.shape[0] if tiled_n is None else tiled_n
     dev = x.device
     y = _gemm_out(M, N, out, dev)
     dynamic = (g_a is None) if compute_global_scale is None else bool(compute_global_scale)
@@ -264,7 +291,8 @@ def nvfp4_linear_decode(x, w_codes, w_scales, g_w, *, hadamard: int = 0, g_a=Non
     elif workspace is False:
         workspace = None
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check("nvfp4_linear_decode", lib().nvfp4_linear_decode(
+    fn = "nvfp4_linear_decode" if tiled_n is None else "nvfp4_linear_decode_tiled"
+    _check(fn, getattr(lib(), fn)(
         _ptr(x), M, K, x.stride(0), hadamard, int(dynamic), _ptr(g_a), _ptr(w_codes), _ptr(w_scales), _ptr(g_w),
         _ptr(y), N, y.stride(0), _ptr(workspace), wsb, _stream(stream)))
     return y, g_a
@@ -325,14 +353,16 @@ class QuantizedWeight:
     hadamard: int
     N: int
     K: int
+    tiled: torch.Tensor | None = None  # NVFP4 codes in the decode GEMM's tile order (optional)
 
 
-def prepare_weight(w: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0) -> QuantizedWeight:
+def prepare_weight(w: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0, tiled: bool = False) -> QuantizedWeight:
     """Quantise a bf16 weight [N, K] once, offline; with hadamard the rotation is folded into it,
-    so y = (x H)(W H)^T = x W^T needs only the online rotation of the activations."""
+    so y = (x H)(W H)^T = x W^T needs only the online rotation of the activations.  tiled
+    (NVFP4): also keep the codes in tile order, which decode-sized calls then stream."""
     if fmt == "nvfp4":
         c, s, g = nvfp4_quantize(w, hadamard)
-        return QuantizedWeight("nvfp4", c, s, g, hadamard, w.shape[0], w.shape[1])
+        return QuantizedWeight("nvfp4", c, s, g, hadamard, w.shape[0], w.shape[1], tile_weights(c) if tiled else None)
     c, s = mxfp4_quantize(w, hadamard)
     return QuantizedWeight("mxfp4", c, s, None, hadamard, w.shape[0], w.shape[1])
 
@@ -398,6 +428,9 @@ def nvfp4_linear(x: torch.Tensor, w: QuantizedWeight, *, out=None, stream=None) 
     """y = x W^T: online (rotated) NVFP4 quantisation of x, then the block-scaled GEMM (for M <= 16
     one fused launch that quantises inside the GEMM; the same result)."""
     if x.shape[0] <= 16 and x.shape[1] % 64 == 0:
+        if w.tiled is not None:
+            return nvfp4_linear_decode(x, w.tiled, w.scales, w.g, hadamard=w.hadamard, out=out, stream=stream,
+                                       tiled_n=w.N)[0]
         return nvfp4_linear_decode(x, w.codes, w.scales, w.g, hadamard=w.hadamard, out=out, stream=stream)[0]
     c, s, g = nvfp4_quantize(x, w.hadamard, stream=stream)
     return nvfp4_gemm(c, s, g, w.codes, w.scales, w.g, out=out, stream=stream)

@@ -230,7 +230,7 @@ template <class C>
 int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const uint8_t *a_codes,
                     const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes, const uint8_t *w_scales,
                     const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy, float *ws,
-                    cudaStream_t st, const QuantOut &qo, const FuseIn *fi = nullptr)
+                    cudaStream_t st, const QuantOut &qo, const FuseIn *fi = nullptr, const uint8_t *a_tiled = nullptr)
 {
     {
         std::lock_guard<std::mutex> lk(g_mutex);
@@ -242,7 +242,8 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
         }
     }
     CUtensorMap tmA, tmB;
-    if (!make_code_map(&tmA, a_codes, M, K, 128))
+    // with tiled A the map is not used; it is built over the tiled buffer so it stays valid
+    if (!make_code_map(&tmA, a_tiled ? a_tiled : a_codes, a_tiled ? (M + 127) / 128 * 128 : M, K, 128))
         return FP4LIN_ERR_CUDA;
     if (fi)
         tmB = tmA;  // not used: the kernel quantises the activations itself
@@ -273,6 +274,7 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
     p.qg = qo.qg;
     p.qhad = qo.qhad;
     p.qkatoms = qo.qkatoms;
+    p.a_tiled = a_tiled;
     if (fi) {
         p.xa = reinterpret_cast<const __nv_bfloat16 *>(fi->x);
         p.ld_xa = fi->ld;
@@ -368,9 +370,12 @@ int launch_gemm_pair(DeviceInfo *dev, int slot, const uint8_t *a_codes, const ui
 
 int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
                const uint8_t *w_scales, const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
-               void *workspace, size_t workspace_bytes, void *stream, const QuantOut &qo = QuantOut{})
+               void *workspace, size_t workspace_bytes, void *stream, const QuantOut &qo = QuantOut{},
+               bool w_tiled = false)
 {
     const bool quant = qo.qc != nullptr;
+    if (w_tiled && M > 16)  // the tile-order weights serve the decode (swapped) form only
+        return (M < 1 || !a_codes) ? FP4LIN_ERR_INVALID_ARGUMENT : FP4LIN_ERR_UNSUPPORTED_SHAPE;
     if (!a_codes || !a_scales || !w_codes || !w_scales || (!y && !quant) || (nv && (!g_a || !g_w)))
         return FP4LIN_ERR_INVALID_ARGUMENT;
     if (quant && (!qo.qs || !qo.qg || (qo.qhad != 0 && qo.qhad != 16)))
@@ -399,7 +404,8 @@ int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const f
     if (pl.swap) {  // the weights take the MMA's M side: operands and shapes swap places
         if (nv)
             return launch_gemm_cfg<GemmCfg<16, true, true>>(dev, 4, pl, w_codes, w_scales, g_w, a_codes, a_scales,
-                                                            g_a, y, N, M, K, ldy, ws, s, qo);
+                                                            g_a, y, N, M, K, ldy, ws, s, qo, nullptr,
+                                                            w_tiled ? w_codes : nullptr);
         return launch_gemm_cfg<GemmCfg<16, false, true>>(dev, 5, pl, w_codes, w_scales, nullptr, a_codes, a_scales,
                                                          nullptr, y, N, M, K, ldy, ws, s, qo);
     }
@@ -674,6 +680,14 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a
                       workspace_bytes, stream);
 }
 
+int nvfp4_gemm_tiled(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_tiled,
+                     const uint8_t *w_scales, const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
+                     void *workspace, size_t workspace_bytes, void *stream)
+{
+    return gemm_entry(true, a_codes, a_scales, g_a, w_tiled, w_scales, g_w, y, M, N, K, ldy, workspace,
+                      workspace_bytes, stream, QuantOut{}, true);
+}
+
 size_t kv_attention_workspace_bytes(int B, int H, int G, int64_t L, int D)
 {
     if (B < 1 || H < 1 || G < 1 || L < 1 || D < 1)
@@ -761,9 +775,10 @@ size_t nvfp4_linear_decode_workspace_bytes(int64_t M, int64_t N, int64_t K)
     return AMAX_MAX_BLOCKS * sizeof(float) + plan_decode(M, N, K, sms).ws_bytes;
 }
 
-int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int hadamard, int compute_global_scale,
-                        float *g_a, const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w, void *y,
-                        int64_t N, int64_t ldy, void *workspace, size_t workspace_bytes, void *stream)
+static int linear_decode_entry(const void *x, int64_t M, int64_t K, int64_t ld_x, int hadamard,
+                               int compute_global_scale, float *g_a, const uint8_t *w_codes, bool tiled,
+                               const uint8_t *w_scales, const float *g_w, void *y, int64_t N, int64_t ldy,
+                               void *workspace, size_t workspace_bytes, void *stream)
 {
     if (!x || !g_a || !w_codes || !w_scales || !g_w || !y)
         return FP4LIN_ERR_INVALID_ARGUMENT;
@@ -810,7 +825,50 @@ int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int h
     }
     // swapped form: the weights are the MMA's M side; g_w's slot carries the activations' scale
     return launch_gemm_cfg<GemmCfg<16, true, true, true>>(dev, 6, pl, w_codes, w_scales, g_w, nullptr, nullptr, g_a,
-                                                           y, N, M, K, ldy, ws, s, QuantOut{}, &fi);
+                                                           y, N, M, K, ldy, ws, s, QuantOut{}, &fi,
+                                                           tiled ? w_codes : nullptr);
+}
+
+int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int hadamard, int compute_global_scale,
+                        float *g_a, const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w, void *y,
+                        int64_t N, int64_t ldy, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return linear_decode_entry(x, M, K, ld_x, hadamard, compute_global_scale, g_a, w_codes, false, w_scales, g_w, y,
+                               N, ldy, workspace, workspace_bytes, stream);
+}
+
+int nvfp4_linear_decode_tiled(const void *x, int64_t M, int64_t K, int64_t ld_x, int hadamard,
+                              int compute_global_scale, float *g_a, const uint8_t *w_tiled, const uint8_t *w_scales,
+                              const float *g_w, void *y, int64_t N, int64_t ldy, void *workspace,
+                              size_t workspace_bytes, void *stream)
+{
+    return linear_decode_entry(x, M, K, ld_x, hadamard, compute_global_scale, g_a, w_tiled, true, w_scales, g_w, y,
+                               N, ldy, workspace, workspace_bytes, stream);
+}
+
+size_t fp4lin_tiled_weight_bytes(int64_t N, int64_t K)
+{
+    if (N < 1 || K < 1)
+        return 0;
+    return (size_t)((N + 127) / 128 * 128) * (size_t)((K + 255) / 256 * 128);
+}
+
+int fp4lin_tile_weights(const uint8_t *codes, int64_t N, int64_t K, uint8_t *tiled, void *stream)
+{
+    if (!codes || !tiled || N < 1 || K < 1)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (K % 64 != 0 || N > INT32_MAX / 2 || K > INT32_MAX / 2)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(codes, 16) || !aligned(tiled, 16))
+        return FP4LIN_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    const int64_t chunks = (int64_t)(fp4lin_tiled_weight_bytes(N, K) / 16);
+    const unsigned grid = (unsigned)std::min<int64_t>((chunks + 255) / 256, (int64_t)dev->sms * 16);
+    weight_tile_kernel<<<grid, 256, 0, as_stream(stream)>>>(codes, N, K, tiled, chunks);
+    return launch_status();
 }
 
 int nvfp4_gemm_quant(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,

@@ -283,6 +283,10 @@ struct GemmParams {
     // maxima at xpart (xnpart > 0) or by every CTA over all the activations (xnpart < 0).
     const __nv_bfloat16 *xa;
     int64_t ld_xa;
+    // A operand in tile order (non-null: loaded by plain bulk copies instead of TMA): tile
+    // (mt, kt) -- 128 rows x 128 code bytes, already in the 128-byte-swizzled image the MMA
+    // reads -- is the 16 KB at ((mt * nk + kt) * 16384).  For decode weights, prepared once.
+    const uint8_t *a_tiled;
     int xhad;
     const float *xpart;
     int xnpart;
@@ -486,7 +490,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + C::RT));
                     armed |= 1u << stage;
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
-                    tma_load_2d(sA, &tmA, &full[stage], kt * 128, mt * C::BM);
+                    if (p.a_tiled)
+                        bulk_load(sA, p.a_tiled + ((int64_t)mt * p.nk + kt) * C::A_BYTES, C::A_BYTES, &full[stage]);
+                    else
+                        tma_load_2d(sA, &tmA, &full[stage], kt * 128, mt * C::BM);
                     const int64_t ka = (int64_t)kt * C::APK;
                     bulk_load(sSFA, p.sfa + ((int64_t)mt * p.katoms + ka) * 512, atoms * 512, &full[stage]);
                     if constexpr (!C::FUSEQ) {
@@ -945,6 +952,26 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *ws, int
             if ((lane & 3) == 0)
                 qo.qs[tc_offset(m, n / 16, qo.qkatoms)] = (uint8_t)sf;
         }
+    }
+}
+
+// Weights [N, K/2] codes -> tile order for the decode GEMM: tile (mt, kt) holds rows
+// 128 mt .. +127, code bytes 128 kt .. +127, as the 128-byte-swizzled image (16-byte chunk c
+// of row r at chunk c ^ (r % 8)); rows past N and bytes past K/2 are zero.  One thread per
+// 16-byte chunk of the output.
+__global__ void __launch_bounds__(256) weight_tile_kernel(const uint8_t *codes, int64_t N, int64_t K, uint8_t *tiled,
+                                                          int64_t chunks)
+{
+    const int64_t nk = (K + 255) / 256;
+    for (int64_t o = (int64_t)blockIdx.x * 256 + threadIdx.x; o < chunks; o += (int64_t)gridDim.x * 256) {
+        const int64_t tile = o >> 10, within = o & 1023;
+        const int r = (int)(within >> 3), c = (int)(within & 7) ^ (r & 7);
+        const int64_t mt = tile / nk, kt = tile - mt * nk;
+        const int64_t row = mt * 128 + r, byte = kt * 128 + c * 16;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row < N && byte < K / 2)  // K % 64 == 0: a 16-byte chunk is all in or all out
+            v = ld_nc_v4(codes + row * (K / 2) + byte);
+        reinterpret_cast<uint4 *>(tiled)[o] = v;
     }
 }
 

@@ -23,7 +23,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported():
     names = header_functions()
-    assert len(names) == 23, names
+    assert len(names) == 27, names
     L = fl.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -132,6 +132,17 @@ def test_gptq_argument_checks():
     assert q(wsp=None) == INVALID
     assert L.mxfp4_gptq_quantize(P, 64, 128, 128, 16, P, 128, P, P, P, ws, None) == INVALID  # 32 or 0
     assert L.mxfp4_gptq_quantize(P, 64, 96, 96, 32, P, 96, P, P, P, ws, None) == SHAPE
+
+
+def test_tiled_weight_checks():
+    L = fl.lib()
+    assert L.fp4lin_tiled_weight_bytes(200, 320) == 256 * 256  # rows to 128, K to 256 values
+    assert L.fp4lin_tiled_weight_bytes(0, 64) == 0
+    assert L.fp4lin_tile_weights(None, 16, 64, P, None) == INVALID
+    assert L.fp4lin_tile_weights(P, 16, 96, P, None) == SHAPE
+    assert L.fp4lin_tile_weights(P, 16, 64, P + 8, None) == MISALIGNED
+    assert L.nvfp4_gemm_tiled(P, P, P, P, P, P, P, 17, 64, 128, 64, None, 0, None) == SHAPE  # decode sizes only
+    assert L.nvfp4_linear_decode_tiled(P, 17, 128, 128, 0, 0, P, P, P, P, P, 64, 64, P, 8192, None) == SHAPE
 
 
 def test_linear_decode_argument_checks():

@@ -96,3 +96,60 @@ def test_linear_routes_decode_sizes_through_fused_path():
     status_ok()
     ca, sa, ga = fl.nvfp4_quantize(x, 16)
     assert torch.equal(_bits(y), _bits(fl.nvfp4_gemm(ca, sa, ga, w.codes, w.scales, w.g)))
+
+
+# ---------------------------------------------------------------- weights in tile order
+def _tile_reference(codes: np.ndarray) -> np.ndarray:
+    """The documented tile order, built with numpy: tile (mt, kt) = rows 128 mt.., code bytes
+    128 kt.., 16-byte chunk c of row r at position c ^ (r % 8); zero padding."""
+    N, KB = codes.shape
+    nm, nk = (N + 127) // 128, (KB + 127) // 128
+    pad = np.zeros((nm * 128, nk * 128), dtype=np.uint8)
+    pad[:N, :KB] = codes
+    t = pad.reshape(nm, 128, nk, 8, 16).transpose(0, 2, 1, 3, 4)  # [mt, kt, r, c, 16]
+    out = np.empty_like(t)
+    for r in range(128):
+        for c in range(8):
+            out[:, :, r, c ^ (r % 8)] = t[:, :, r, c]
+    return out.reshape(-1)
+
+
+@pytest.mark.parametrize("N,K", [(200, 320), (128, 256), (1, 64), (4096, 1088)])
+def test_tile_order_matches_documented_layout(N, K):
+    codes = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=DEV)
+    tiled = fl.tile_weights(codes)
+    status_ok()
+    assert np.array_equal(tiled.cpu().numpy(), _tile_reference(codes.cpu().numpy()))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 640, 256), (5, 320, 1088), (16, 14336, 512), (16, 4096, 4096), (4, 136, 64),
+                                   (16, 4096, 14336)])
+@pytest.mark.parametrize("hadamard", [0, 16])
+def test_tiled_weights_give_the_same_bits(M, N, K, hadamard):
+    x = si.student_t_bf16(M * 5 + K, M, K).to(DEV)
+    cw, sw, gw = _weights(N, K, hadamard, N + 2 * K)
+    tiled = fl.tile_weights(cw)
+    ca, sa, ga = fl.nvfp4_quantize(x, hadamard)
+    y_ref = fl.nvfp4_gemm(ca, sa, ga, cw, sw, gw)
+    status_ok()
+    y_t = fl.nvfp4_gemm_tiled(ca, sa, ga, tiled, sw, gw, N)
+    y_f, g = fl.nvfp4_linear_decode(x, tiled, sw, gw, hadamard=hadamard, tiled_n=N)
+    status_ok()
+    assert torch.equal(_bits(y_t), _bits(y_ref))
+    assert torch.equal(_bits(y_f), _bits(y_ref))
+    assert torch.equal(g, ga)
+    y_u, _ = fl.nvfp4_linear_decode(x, tiled, sw, gw, hadamard=hadamard, tiled_n=N, workspace=False,
+                                    g_a=ga.clone())  # unsplit, static scale
+    status_ok()
+    assert torch.equal(_bits(y_u), _bits(y_ref))
+
+
+def test_linear_uses_tiled_weights():
+    M, N, K = 3, 1024, 512
+    x = si.student_t_bf16(60, M, K).to(DEV)
+    wt = fl.prepare_weight(si.normal_bf16(61, N, K, std=0.02).to(DEV), "nvfp4", 16, tiled=True)
+    assert wt.tiled is not None
+    y = fl.nvfp4_linear(x, wt)
+    status_ok()
+    ca, sa, ga = fl.nvfp4_quantize(x, 16)
+    assert torch.equal(_bits(y), _bits(fl.nvfp4_gemm(ca, sa, ga, wt.codes, wt.scales, wt.g)))
