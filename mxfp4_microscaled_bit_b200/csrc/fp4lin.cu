@@ -200,12 +200,11 @@ int raster_group(int num_mt)
 // Launch with programmatic stream serialisation: the kernel may start before the previous one
 // in the stream has finished, and must pdl_wait before touching anything that one writes.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
-                       Args &&...args)
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args &&...args)
 {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -570,14 +569,22 @@ int nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
         if (launch_status() != FP4LIN_OK)
             return FP4LIN_ERR_CUDA;
     }
+    // with the computed scale the encode pass starts under the amax pass (programmatic
+    // dependent launch): it issues its loads of x first and waits only to read the partials
+    cudaError_t e = cudaSuccess;
     if (hadamard && compute_global_scale)
-        nvfp4_quant_kernel<true, true><<<grid, QTHREADS, 0, s>>>(q, g, partials, n_partials);
+        e = launch_pdl(nvfp4_quant_kernel<true, true>, grid, QTHREADS, 0, s, q, g, (const float *)partials, n_partials);
     else if (hadamard)
         nvfp4_quant_kernel<true, false><<<grid, QTHREADS, 0, s>>>(q, g, partials, 0);
     else if (compute_global_scale)
-        nvfp4_quant_kernel<false, true><<<grid, QTHREADS, 0, s>>>(q, g, partials, n_partials);
+        e = launch_pdl(nvfp4_quant_kernel<false, true>, grid, QTHREADS, 0, s, q, g, (const float *)partials,
+                       n_partials);
     else
         nvfp4_quant_kernel<false, false><<<grid, QTHREADS, 0, s>>>(q, g, partials, 0);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return FP4LIN_ERR_CUDA;
+    }
     if (launch_status() != FP4LIN_OK)
         return FP4LIN_ERR_CUDA;
     return launch_padding(q, dev, s);

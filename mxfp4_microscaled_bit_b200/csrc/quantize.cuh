@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(QTHREADS)
                 raw[u][j] = 0;
     }
     if (DYNAMIC) {
+        pdl_wait();  // launched under the amax pass: its partials are complete past this point
         float m = 0.0f;
         for (int k = threadIdx.x; k < n_partials; k += QTHREADS)
             m = fmaxf(m, partials[k]);
