@@ -73,12 +73,16 @@ __device__ __forceinline__ void kv_fp8_word(uint32_t w, uint32_t s2u, uint32_t *
         : "r"(w), "r"(s2u));
 }
 
-// The block scale / 8 as an f16x2 bit pattern (exact in f16); bit conversions only, no
-// type punning through pointers.
-__device__ __forceinline__ uint32_t kv_scale_half2(uint32_t sf)
+// The block scale / 8 in both halves of an f16x2, from a 16-bit word holding the scale byte
+// twice: the hardware's E4M3 -> f16 conversion (exact: E4M3 is a subset of f16) and an exact
+// multiply by 1/8 (the smallest result, 2^-12, is still a normal f16).
+__device__ __forceinline__ uint32_t kv_scale_pair(uint32_t sf_twice)
 {
-    const uint32_t u = __half_as_ushort(__float2half_rn(__fmul_rn(e4m3_value(sf), 0.125f)));
-    return u | (u << 16);
+    uint32_t h;
+    asm("{\n\t.reg .b16 p;\n\tcvt.u16.u32 p, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, p;\n\tmul.rn.f16x2 %0, %0, %2;\n\t}"
+        : "=r"(h)
+        : "r"(sf_twice), "r"(0x30003000u));  // 0x3000: 0.125 in f16
+    return h;
 }
 
 __device__ __forceinline__ float2 half2_to_float2(uint32_t h)
@@ -217,11 +221,10 @@ __global__ void __launch_bounds__(KA_THREADS, 2) kv_attn_tc_kernel(KvAttnShape a
         float sc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const int blk = 2 * r + (tg >> 1);  // the block of dimensions 32r + 8t .. +7
-            const int sh = 8 * (blk & 3);
+            const uint32_t dup = (uint32_t)(2 * r + (tg >> 1)) * 0x11u;  // scale byte of dimensions 32r + 8t .., twice
             uint32_t ha[4], hb[4];
-            kv_fp8_word(wa[r], kv_scale_half2(((blk < 4 ? sa.x : sa.y) >> sh) & 0xFFu), ha);
-            kv_fp8_word(wb[r], kv_scale_half2(((blk < 4 ? sb.x : sb.y) >> sh) & 0xFFu), hb);
+            kv_fp8_word(wa[r], kv_scale_pair(__byte_perm(sa.x, sa.y, dup)), ha);
+            kv_fp8_word(wb[r], kv_scale_pair(__byte_perm(sb.x, sb.y, dup)), hb);
             mma_16816x(sc, ha[0], hb[0], ha[1], hb[1], qb[2 * r][0], qb[2 * r][1]);
             mma_16816x(sc, ha[2], hb[2], ha[3], hb[3], qb[2 * r + 1][0], qb[2 * r + 1][1]);
         }
@@ -311,7 +314,7 @@ __global__ void __launch_bounds__(KA_THREADS, 2) kv_attn_tc_kernel(KvAttnShape a
                 c = *reinterpret_cast<const uint2 *>(s_vc + rp[e] * (KA_D / 2) + 8 * gq);
                 sfb = s_vs[rp[e] * 8 + gq];
             }
-            const uint32_t s2u = kv_scale_half2(sfb);
+            const uint32_t s2u = kv_scale_pair(sfb * 0x101u);
             kv_fp8_word(c.x, s2u, hv[e]);
             kv_fp8_word(c.y, s2u, hv[e] + 4);
         }
