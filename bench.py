@@ -43,10 +43,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP/s)
 
 # DRAM bytes (read + write) per step for a kernel, from one ncu capture of the current build
-# (profiles/*.md); None where no capture covers the kernel as it stands.
+# (summarised under profiles/); None where no capture covers the kernel as it stands.
 NCU_TRAFFIC = {
-    "gemm": 290.8e6,          # profiles/gemm_nvfp4_prefill_8192x14336x4096.md, one launch
-    "kv_load_fp8": 5.914e9,   # profiles/kv_load_fp8_8x8x32768x128.md: 369.6 MB x 8 (units) x 2 (K, V)
+    "gemm": 290.8e6,          # the 8192x14336x4096 prefill GEMM, one launch
+    "kv_load_fp8": 5.914e9,   # 369.6 MB per 8x8x32768x128 cache, x 8 (units) x 2 (K, V)
     "quantize": None,         # the capture covers the quantise pass only, not the amax pass
     "kv_store": None,
 }

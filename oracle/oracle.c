@@ -21,7 +21,7 @@
  *   [MRGPTQ]  the MR-GPTQ abstract (hyper.ai/de/papers/2509.23202), "Abstract".
  *   [KV]      the NVFP4 KV-cache story (hyper.ai/de/stories/...).
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent, garbled or in conflict:
  *   R1 E2M1 has exponent bias 1 (the pages give "about -6 to 6", which with
  *      1 sign / 2 exponent / 1 mantissa bit forces bias 1); encoding rounds to
  *      nearest, ties to the even code, saturates at 6, keeps the sign of zero.
