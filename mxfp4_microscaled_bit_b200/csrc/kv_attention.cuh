@@ -23,9 +23,9 @@
 namespace fp4lin {
 
 constexpr int KA_D = 128;          // head dimension
-constexpr int KA_THREADS = 256;
+constexpr int KA_THREADS = 128;  // four warps: four CTAs share an SM, so one loads while others compute
 constexpr int KA_WARPS = KA_THREADS / 32;
-constexpr int KA_CHUNK = 512;      // positions per CTA
+constexpr int KA_CHUNK = 256;      // positions per CTA
 constexpr int KA_GMAX = 8;         // query heads per kv head
 constexpr int KA_SBUF = KA_CHUNK > KA_WARPS * KA_D ? KA_CHUNK : KA_WARPS * KA_D;  // score / output floats per head
 
@@ -142,7 +142,7 @@ __device__ __forceinline__ uint32_t prmt_hi(uint32_t x, uint32_t y)
 // lane needs 16 contiguous dimensions (8 code bytes, one scale) of each of its 4 rows; prmt
 // pairs two rows' values into one fragment register.
 template <int G>
-__global__ void __launch_bounds__(KA_THREADS, 2) kv_attn_tc_kernel(KvAttnShape a)
+__global__ void __launch_bounds__(KA_THREADS, 4) kv_attn_tc_kernel(KvAttnShape a)
 {
     extern __shared__ __align__(128) uint8_t ka_smem[];
     uint8_t *s_kc = ka_smem;
