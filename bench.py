@@ -208,23 +208,27 @@ class Workload:
         assert self.fl.device_status() == 0
         self.setup_s["kv"] = time.time() - t0
 
-    def step(self, ev=None):
-        """One pass of the hot path; `ev` (5 CUDA events) brackets its four parts."""
+    def step(self, ev=None, A=None, y=None, kv_new=None):
+        """One pass of the hot path; `ev` (5 CUDA events) brackets its four parts.  A, y, kv_new:
+        other buffers of the same shapes in place of the workload's own."""
         fl = self.fl
+        A = self.A if A is None else A
+        y = self.y if y is None else y
+        kv_new = self.kv_new if kv_new is None else kv_new
         if ev is not None:
             ev[0].record()
-        fl.nvfp4_quantize(self.A, 16, self.g_a, compute_global_scale=True, codes=self.a_codes,
+        fl.nvfp4_quantize(A, 16, self.g_a, compute_global_scale=True, codes=self.a_codes,
                           scales=self.a_scales, workspace=self.q_ws)
         if ev is not None:
             ev[1].record()
-        fl.nvfp4_gemm(self.a_codes, self.a_scales, self.g_a, self.w.codes, self.w.scales, self.w.g, out=self.y,
+        fl.nvfp4_gemm(self.a_codes, self.a_scales, self.g_a, self.w.codes, self.w.scales, self.w.g, out=y,
                       workspace=False)
         if ev is not None:
             ev[2].record()
         if self.with_kv:
             for which in ("k", "v"):
                 codes, scales, _, _ = self.cache[which]
-                fl.kv_nvfp4_store(self.kv_new[which], self.pos, self.kv_g[which], codes, scales)
+                fl.kv_nvfp4_store(kv_new[which], self.pos, self.kv_g[which], codes, scales)
             if ev is not None:
                 ev[3].record()
             for which in ("k", "v"):
@@ -581,7 +585,48 @@ def main():
         e2e_full()
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = time_loop(e2e_full, args.e2e_steps, stream) / args.e2e_steps
+    e2e_serial_ms = time_loop(e2e_full, args.e2e_steps, stream) / args.e2e_steps
+    e2e_serial_ms = max_over_ranks(e2e_serial_ms, dev)
+
+    # ---- the same, pipelined as a serving loop would run it: two sets of device buffers; each
+    #      step's copies in (A, the new K/V rows) and out (y, the FP8 output scales) run on copy
+    #      streams, overlapping the neighbouring steps' compute; every copy stays in the timed region
+    A_dev = [w.A, torch.empty_like(w.A)]
+    y_dev = [w.y, torch.empty_like(w.y)]
+    kv_dev = [w.kv_new, {k: torch.empty_like(v) for k, v in w.kv_new.items()}]
+    y_host = [w.y_host, torch.empty(w.y.shape, dtype=w.y.dtype, pin_memory=True)]
+    osc_host = [torch.empty(2, dtype=torch.float32, pin_memory=True) for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in, ev_done, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+
+    def e2e_pipelined(n):
+        s_in.wait_stream(stream)
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[b])  # buffers b were read by step i - 2
+                A_dev[b].copy_(w.A_host, non_blocking=True)
+                for which in ("k", "v"):
+                    kv_dev[b][which].copy_(w.kv_new_host[which], non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])  # y of step i - 2 has left the device
+            w.step(A=A_dev[b], y=y_dev[b], kv_new=kv_dev[b])
+            ev_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                y_host[b].copy_(y_dev[b], non_blocking=True)
+                osc_host[b][0:1].copy_(w.cache["k"][3], non_blocking=True)
+                osc_host[b][1:2].copy_(w.cache["v"][3], non_blocking=True)
+                ev_out[b].record(s_out)
+        stream.wait_stream(s_out)
+
+    e2e_pipelined(2)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = time_loop(lambda: e2e_pipelined(args.e2e_steps), 1, stream) / args.e2e_steps
     e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = w.A.numel() * 2 + sum(w.kv_new[k].numel() * 2 for k in ("k", "v"))
     d2h = w.y.numel() * 2 + 8
@@ -679,7 +724,10 @@ def main():
                         "note": "y handed on as NVFP4 (static g_y, H16): nvfp4_gemm + nvfp4_quantize vs "
                                 "nvfp4_gemm_quant without bf16 y; back-to-back calls, operands L2-warm"}},
         "e2e": {"value": ws * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "serial_ms_per_step": e2e_serial_ms,
+                "note": "public API, pinned host buffers; copies of step i+1 in and step i-1 out overlap step i "
+                        "(two device buffer sets); serial_ms_per_step: the same with copy, step, copy in sequence"},
         "gpu_launches": Workload.LAUNCHES_PER_STEP * args.steps,
         "clocks": clk,
         "peaks": {**peaks, "source": peak_src},
