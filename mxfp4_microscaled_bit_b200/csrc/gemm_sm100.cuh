@@ -374,8 +374,9 @@ __device__ __forceinline__ void tile_coords(const GemmParams &p, int64_t w, int 
 // of every k-tile.  fuseq_load fetches its 16 bf16 values (nothing outside the activations);
 // fuseq_store quantises them into the stage: the 8 code bytes at their place in the
 // 128-byte-swizzled 16-row operand tile (16-byte chunk index XOR row % 8), the scale byte at
-// its place in the stage's scale atoms; blocks outside the activations get zeros.  The same
-// arithmetic as nvfp4_quant_kernel, so the codes and scales are those it would write.
+// its place in the row's scale lines (fuseq_store); blocks outside the activations get
+// zeros.  The same arithmetic as nvfp4_quant_kernel, so the codes and scales are those it
+// would write.
 struct FuseRaw {
     uint4 u0, u1;
 };
@@ -413,7 +414,11 @@ __device__ __forceinline__ void fuseq_store(const GemmParams &p, uint8_t *sB, ui
         hi = pack_e2m1x8(v + 8);
     }
     *reinterpret_cast<uint2 *>(sB + r * 128 + (((c >> 1) ^ (r & 7)) << 4) + ((c & 1) << 3)) = make_uint2(lo, hi);
-    sSFB[(c >> 2) * 512 + r * 16 + (c & 3)] = (uint8_t)sf;
+    // two k-blocks' scales per 16-byte line of row r: k-blocks 2h and 2h+1 at bytes 0..3 and
+    // 8..11 of line r of the 512-byte region h, so one copy serves two MMAs, which read their
+    // scales at TMEM column offsets 0 and 2 of it (offsets the 64-row B tiles use as well)
+    const int kb = c >> 2;
+    sSFB[(kb >> 1) * 512 + r * 16 + (kb & 1) * 8 + (c & 3)] = (uint8_t)sf;
 }
 
 // k-tiles whose activations are fetched ahead of the one being encoded
@@ -553,15 +558,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         const int a = C::NV ? kb : kb >> 1;
                         if (C::NV || (kb & 1) == 0) {
                             tc_cp_atom(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
+                            if constexpr (C::FUSEQ) {  // one copy per two k-blocks (see fuseq_store)
+                                if ((kb & 1) == 0)
+                                    tc_cp_atom(tm_sfb + (kb >> 1) * 4, desc_sf_atom(smem_u32(sSFB + (kb >> 1) * 512)));
+                            } else {
 #pragma unroll
-                            for (int rt = 0; rt < C::RT; ++rt)
-                                tc_cp_atom(tm_sfb + a * C::RT * 4 + rt * 4,
-                                           desc_sf_atom(smem_u32(sSFB + (rt * C::APK + a) * 512)));
+                                for (int rt = 0; rt < C::RT; ++rt)
+                                    tc_cp_atom(tm_sfb + a * C::RT * 4 + rt * 4,
+                                               desc_sf_atom(smem_u32(sSFB + (rt * C::APK + a) * 512)));
+                            }
                         }
                         uint32_t sfa, sfb, idesc;
                         if (C::NV) {
                             sfa = tm_sfa + kb * 4;
-                            sfb = tm_sfb + kb * C::RT * 4 + sfb_off;
+                            // rows n < 32 of B read their scales at lane n, column 0 of the address:
+                            // k-block kb's scales sit at column 4 (kb / 2) + 2 (kb % 2)
+                            sfb = C::FUSEQ ? tm_sfb + (kb >> 1) * 4 + (kb & 1) * 2
+                                           : tm_sfb + kb * C::RT * 4 + sfb_off;
                             idesc = C::IDESC;
                         } else {
                             const uint32_t byte = (uint32_t)(kb & 1) * 2u;  // second MMA of an atom: scale bytes 2..3
