@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
                 "oracle_kv_load_fp8": (None, [u8p, u8p, i64, ctypes.c_int, ctypes.c_int, i64, ctypes.c_int, u8p]),
                 "oracle_gptq": (None, [u16p, i64, i64, i64, ctypes.c_int, ctypes.c_int, f32p, ctypes.c_float, u8p,
                                        u8p, f32p]),
+                "oracle_gptq_mse": (None, [u16p, i64, i64, i64, ctypes.c_int, f32p, ctypes.c_float, u8p, u8p, f32p]),
                 "oracle_kv_attention": (None, [u16p, u8p, u8p, ctypes.c_float, u8p, u8p, ctypes.c_float, i64,
                                                ctypes.c_int, ctypes.c_int, ctypes.c_int, i64, ctypes.c_int, f64p]),
             }
@@ -205,11 +206,12 @@ def mxfp4_quantize(x, hadamard: int = 0, nearest: bool = False):
     return codes, sf
 
 
-def gptq(w, u: np.ndarray, fmt: str = "nvfp4", hadamard: int = 0, g=None, want_err: bool = False):
+def gptq(w, u: np.ndarray, fmt: str = "nvfp4", hadamard: int = 0, g=None, want_err: bool = False,
+         mse: bool = False):
     """MR-GPTQ (reading R12) of bf16 weights w [N, K] with the inverse-Hessian factor u
     (fp32 [K, K], upper triangle read).  -> (codes [N, K/2], sf [N, K/G] row-major, g
     (NVFP4; None for MXFP4)[, err fp32 [N, K]]).  NVFP4's g defaults to the rotated w's
-    tensor scale, as nvfp4_quantize computes it."""
+    tensor scale, as nvfp4_quantize computes it.  mse (NVFP4): block scales by R9."""
     wb = _bits(w)
     N, K = wb.shape
     uu = np.ascontiguousarray(u, dtype=np.float32)
@@ -220,9 +222,15 @@ def gptq(w, u: np.ndarray, fmt: str = "nvfp4", hadamard: int = 0, g=None, want_e
     codes = np.zeros((N, K // 2), dtype=np.uint8)
     sf = np.zeros((N, K // group), dtype=np.uint8)
     err = np.zeros((N, K), dtype=np.float32) if want_err else None
-    lib().oracle_gptq(_p(wb, ctypes.c_uint16), N, K, K, group, hadamard, _p(uu, ctypes.c_float),
-                      float(g) if fmt == "nvfp4" else 1.0, _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8),
-                      _p(err, ctypes.c_float) if want_err else None)
+    if mse:
+        assert fmt == "nvfp4"
+        lib().oracle_gptq_mse(_p(wb, ctypes.c_uint16), N, K, K, hadamard, _p(uu, ctypes.c_float), float(g),
+                              _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8),
+                              _p(err, ctypes.c_float) if want_err else None)
+    else:
+        lib().oracle_gptq(_p(wb, ctypes.c_uint16), N, K, K, group, hadamard, _p(uu, ctypes.c_float),
+                          float(g) if fmt == "nvfp4" else 1.0, _p(codes, ctypes.c_uint8), _p(sf, ctypes.c_uint8),
+                          _p(err, ctypes.c_float) if want_err else None)
     out = (codes, sf, np.float32(g) if fmt == "nvfp4" else None)
     return out + (err,) if want_err else out
 

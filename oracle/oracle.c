@@ -65,7 +65,10 @@
  *      the format's own rule (R3 with the static tensor scale g of the
  *      rotated W, or R4); q = the dequantised code; e = (w_j - q) / U[j][j];
  *      then w_k <- fma(-e, U[j][k], w_k) for every k > j, in binary32, so each
- *      value receives its corrections one at a time in increasing j.
+ *      value receives its corrections one at a time in increasing j.  Variant
+ *      (NVFP4): the block scale chosen by R9 (least squared error over all 127
+ *      E4M3 codes) from the block's current values, the abstract's
+ *      format-specific optimisation read as the format's best scale.
  */
 #include <math.h>
 #include <stdint.h>
@@ -407,8 +410,8 @@ EXPORT void oracle_mxfp4_quantize_nearest(const uint16_t *x, int64_t rows, int64
  * group: 16 (NVFP4, E4M3 scales relative to g) or 32 (MXFP4, E8M0 scales).
  * codes [N, K/2] (R6); sf [N, K/group] row-major; err [N, K] (optional): the
  * scaled errors e, the quantities GPTQ feeds back. */
-EXPORT void oracle_gptq(const uint16_t *w, int64_t N, int64_t K, int64_t ld, int group, int hadamard,
-                        const float *u, float g, uint8_t *codes, uint8_t *sf, float *err)
+static void gptq_sweep(const uint16_t *w, int64_t N, int64_t K, int64_t ld, int group, int hadamard,
+                       const float *u, float g, int mse, uint8_t *codes, uint8_t *sf, float *err)
 {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t n = 0; n < N; ++n) {
@@ -422,9 +425,10 @@ EXPORT void oracle_gptq(const uint16_t *w, int64_t N, int64_t K, int64_t ld, int
                 for (int i = 0; i < group; ++i)
                     if (fabsf(row[j + i]) > amax)
                         amax = fabsf(row[j + i]);
-                if (group == 16) { /* R3 */
+                if (group == 16) { /* R3, or R9 with mse */
+                    uint8_t scratch[16];
                     float t = (amax / 6.0f) / g;
-                    uint8_t s = oracle_e4m3_encode(t);
+                    uint8_t s = mse ? nvfp4_block_mse(row + j, g, scratch) : oracle_e4m3_encode(t);
                     d = (float)oracle_e4m3_decode(s) * g;
                     rcp = (d > 0.0f) ? 1.0f / d : 0.0f;
                     sf[n * (K / 16) + j / 16] = s;
@@ -456,6 +460,19 @@ EXPORT void oracle_gptq(const uint16_t *w, int64_t N, int64_t K, int64_t ld, int
         }
         free(row);
     }
+}
+
+EXPORT void oracle_gptq(const uint16_t *w, int64_t N, int64_t K, int64_t ld, int group, int hadamard,
+                        const float *u, float g, uint8_t *codes, uint8_t *sf, float *err)
+{
+    gptq_sweep(w, N, K, ld, group, hadamard, u, g, 0, codes, sf, err);
+}
+
+/* MR-GPTQ with R9's MSE-optimal NVFP4 block scales (group 16). */
+EXPORT void oracle_gptq_mse(const uint16_t *w, int64_t N, int64_t K, int64_t ld, int hadamard, const float *u,
+                            float g, uint8_t *codes, uint8_t *sf, float *err)
+{
+    gptq_sweep(w, N, K, ld, 16, hadamard, u, g, 1, codes, sf, err);
 }
 
 /* ------------------------------------------------------------------ scale layout (R7) */

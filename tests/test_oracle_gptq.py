@@ -152,3 +152,38 @@ def test_gptq_beats_rounding_on_correlated_inputs(orc, fmt, had):
 
     e_gptq, e_rtn = out_err(codes, sf), out_err(rc, rs)
     assert e_gptq < 0.8 * e_rtn, (e_gptq, e_rtn)
+
+
+# ---------------------------------------------------------------- the MSE-scale variant (R12 with R9)
+@pytest.mark.parametrize("had", [0, 16])
+def test_mse_variant_identity_hessian_is_the_mse_quantiser(orc, had):
+    N, K = 16, 128
+    w = si.normal_bf16(4, N, K, std=0.02)
+    codes, sf, g = orc.gptq(w, np.eye(K, dtype=np.float32), "nvfp4", had, mse=True)
+    rc, rs, _ = orc.nvfp4_quantize_mse(w, had, g)
+    assert np.array_equal(codes, rc) and np.array_equal(sf, rs)
+
+
+def test_mse_variant_sweep_identity(orc):
+    N, K = 12, 128
+    w = si.normal_bf16(23, N, K, std=0.02)
+    u = orc.gptq_hessian_factor(si.gptq_calibration(24, 3 * K, K), 16)
+    codes, sf, g, err = orc.gptq(w, u, "nvfp4", 16, want_err=True, mse=True)
+    assert _sweep_identity_residual(orc, _rotated_f32(orc, w, 16), codes, sf, g, "nvfp4", err, u) < 1e-4
+
+
+def test_mse_variant_lowers_output_error(orc):
+    N, K = 64, 256
+    w = si.normal_bf16(33, N, K, std=0.02)
+    x = si.gptq_calibration(34, 4 * K, K)
+    u = orc.gptq_hessian_factor(x, 16)
+    R = orc.hadamard_matrix(16).astype(np.float64) / 4.0
+    xr = (x.reshape(x.shape[0], K // 16, 16) @ R.T).reshape(x.shape)
+    w_rot = _rotated_f32(orc, w, 16).astype(np.float64)
+
+    def out_err(c, s, g):
+        return np.linalg.norm(xr @ (w_rot - orc.dequant(c, s, "nvfp4", g)).T)
+
+    c0, s0, g0 = orc.gptq(w, u, "nvfp4", 16)
+    c1, s1, g1 = orc.gptq(w, u, "nvfp4", 16, mse=True)
+    assert out_err(c1, s1, g1) < out_err(c0, s0, g0)
