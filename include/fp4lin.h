@@ -348,6 +348,17 @@ int nvfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int h
 int mxfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard,
                         const float *u, int64_t ld_u, uint8_t *codes, uint8_t *scales,
                         void *workspace, size_t workspace_bytes, void *stream);
+/*
+ * nvfp4_gptq_quantize with each 16-value block's scale chosen, from the row's
+ * current values at the block's first column, as nvfp4_quantize_mse chooses it
+ * (least squared error over all 127 E4M3 codes, ties to the smaller code): the
+ * format-specific scale of the MR-GPTQ abstract read as NVFP4's best scale.
+ * Arguments and errors as nvfp4_gptq_quantize; slower (127 candidates per block).
+ */
+int nvfp4_gptq_quantize_mse(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard,
+                            const float *u, int64_t ld_u, int compute_global_scale, float *g,
+                            uint8_t *codes, uint8_t *scales,
+                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Decode weights in tile order.  The decode-sized GEMM (M <= 16) streams the

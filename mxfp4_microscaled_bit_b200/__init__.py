@@ -64,6 +64,7 @@ EXPORTS = {
     "nvfp4_linear_decode_tiled": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64,
                                          _vp, _sz, _vp]),
     "nvfp4_gptq_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "nvfp4_gptq_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_gptq_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_decode": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _sz,
                                    _vp]),
@@ -389,10 +390,12 @@ def gptq_hessian_factor(x: torch.Tensor, hadamard: int = 0, damp: float = 0.01) 
 
 
 def gptq_quantize(w: torch.Tensor, u: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0, g=None, *,
-                  compute_global_scale: bool | None = None, codes=None, scales=None, workspace=None, stream=None):
+                  compute_global_scale: bool | None = None, codes=None, scales=None, workspace=None, stream=None,
+                  mse: bool = False):
     """MR-GPTQ of bf16 weights w [N, K] with the inverse-Hessian factor u [K, K] (float32).
     Returns (codes [N, K/2], scales, g) -- g None for MXFP4 -- ready for nvfp4_gemm /
-    mxfp4_gemm against activations rotated the same way."""
+    mxfp4_gemm against activations rotated the same way.  mse (NVFP4): block scales of least
+    squared error (nvfp4_gptq_quantize_mse)."""
     N, K = w.shape
     dev = w.device
     G = 16 if fmt == "nvfp4" else 32
@@ -407,7 +410,8 @@ def gptq_quantize(w: torch.Tensor, u: torch.Tensor, fmt: str = "nvfp4", hadamard
         dynamic = (g is None) if compute_global_scale is None else bool(compute_global_scale)
         if g is None:
             g = torch.empty(1, dtype=torch.float32, device=dev)
-        _check("nvfp4_gptq_quantize", lib().nvfp4_gptq_quantize(
+        fn = "nvfp4_gptq_quantize_mse" if mse else "nvfp4_gptq_quantize"
+        _check(fn, getattr(lib(), fn)(
             _ptr(w), N, K, w.stride(0), hadamard, _ptr(u), u.stride(0), int(dynamic), _ptr(g), _ptr(codes),
             _ptr(scales), _ptr(workspace), wsb, _stream(stream)))
         return codes, scales, g

@@ -1155,7 +1155,7 @@ struct GptqStreams {
 // Shared by both formats: checks, rotation, the optional tensor scale, the block sweep.
 int gptq_entry(bool nv, const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,
                int64_t ld_u, int compute_global_scale, float *g, uint8_t *codes, uint8_t *scales, void *workspace,
-               size_t workspace_bytes, void *stream)
+               size_t workspace_bytes, void *stream, bool mse = false)
 {
     const int G = nv ? 16 : 32;
     if (!w || !u || !codes || !scales || (nv && !g) || !workspace)
@@ -1248,7 +1248,9 @@ int gptq_entry(bool nv, const void *w, int64_t N, int64_t K, int64_t ld_w, int h
         const int64_t s1 = std::min<int64_t>(K, s0 + GQ_SB), s2 = std::min<int64_t>(K, s1 + GQ_SB);
         a.et = et_base + ((s0 / GQ_SB) & 1) * GQ_SB * a.np;
         for (int64_t c0 = s0; c0 < s1; c0 += GQ_B) {
-            if (nv)
+            if (nv && mse)
+                gptq_block_kernel<true, true><<<bgrid, GQ_ROWS, 0, s>>>(a, c0, s0);
+            else if (nv)
                 gptq_block_kernel<true><<<bgrid, GQ_ROWS, 0, s>>>(a, c0, s0);
             else
                 gptq_block_kernel<false><<<bgrid, GQ_ROWS, 0, s>>>(a, c0, s0);
@@ -1293,6 +1295,14 @@ int nvfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int h
 {
     return gptq_entry(true, w, N, K, ld_w, hadamard, u, ld_u, compute_global_scale, g, codes, scales, workspace,
                       workspace_bytes, stream);
+}
+
+int nvfp4_gptq_quantize_mse(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,
+                            int64_t ld_u, int compute_global_scale, float *g, uint8_t *codes, uint8_t *scales,
+                            void *workspace, size_t workspace_bytes, void *stream)
+{
+    return gptq_entry(true, w, N, K, ld_w, hadamard, u, ld_u, compute_global_scale, g, codes, scales, workspace,
+                      workspace_bytes, stream, true);
 }
 
 int mxfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard, const float *u,

@@ -29,7 +29,7 @@
 // decisions downstream must see exactly the binary32 values the sweep defines.
 #pragma once
 
-#include "quantize.cuh"
+#include "scale_search.cuh"
 
 namespace fp4lin {
 
@@ -123,7 +123,7 @@ __device__ __forceinline__ float e8m0_value(uint32_t byte)
 // Column J of a row's 64-value block: the block scale at the first column of each format
 // block, the code, the error, and the corrections of the later columns.  A template over J
 // so that every index into the register arrays is a constant.
-template <bool NV, int J>
+template <bool NV, bool MSE, int J>
 struct GptqColumn {
     static __device__ __forceinline__ void run(float (&w)[GQ_B], const float (&us)[GQ_B][GQ_B], float g, float &mul,
                                                float &back, uint32_t (&code_words)[GQ_B / 8], uint32_t &sf_word,
@@ -136,7 +136,19 @@ struct GptqColumn {
             for (int i = 0; i < G; ++i)
                 amax = fmaxf(amax, fabsf(w[J + i]));
             uint32_t sf;
-            if constexpr (NV) {
+            if constexpr (NV && MSE) {  // the least squared error over all 127 E4M3 codes (ties: smaller)
+                float best = block_sq_error(&w[J], 0u, g);
+                sf = 0u;
+                for (uint32_t cand = 1; cand <= 126; ++cand) {
+                    const float e = block_sq_error(&w[J], cand, g);
+                    if (e < best) {
+                        best = e;
+                        sf = cand;
+                    }
+                }
+                back = __fmul_rn(e4m3_value(sf), g);
+                mul = back > 0.0f ? __fdiv_rn(1.0f, back) : 0.0f;
+            } else if constexpr (NV) {
                 sf = nvfp4_block_scale(amax, g, mul);
                 back = __fmul_rn(e4m3_value(sf), g);
             } else {
@@ -159,13 +171,14 @@ struct GptqColumn {
         for (int k = J + 1; k < GQ_B; ++k)
             w[k] = __fmaf_rn(-e, us[J][k], w[k]);
         if constexpr (J + 1 < GQ_B)
-            GptqColumn<NV, J + 1>::run(w, us, g, mul, back, code_words, sf_word, ecol, np);
+            GptqColumn<NV, MSE, J + 1>::run(w, us, g, mul, back, code_words, sf_word, ecol, np);
     }
 };
 
 // One 64-column block of the sweep for every row.  NV: NVFP4 (16-value blocks, E4M3 scales
-// relative to *g); else MXFP4 (32-value blocks, E8M0 scales by the OCP exponent rule).
-template <bool NV>
+// relative to *g; MSE: the scale of least squared error over all 127 E4M3 codes, as
+// nvfp4_quant_mse_kernel picks it); else MXFP4 (32-value blocks, E8M0 by the OCP rule).
+template <bool NV, bool MSE = false>
 __global__ void __launch_bounds__(GQ_ROWS) gptq_block_kernel(GptqArgs a, int64_t c0, int64_t s0)
 {
     __shared__ float us[GQ_B][GQ_B];
@@ -191,7 +204,7 @@ __global__ void __launch_bounds__(GQ_ROWS) gptq_block_kernel(GptqArgs a, int64_t
     float mul = 0.0f, back = 0.0f;  // x -> code scale and code -> value scale of the current block
     uint32_t code_words[GQ_B / 8];
     uint32_t sf_word = 0;
-    GptqColumn<NV, 0>::run(w, us, g, mul, back, code_words, sf_word, a.et + (c0 - s0) * a.np + n, a.np);
+    GptqColumn<NV, MSE, 0>::run(w, us, g, mul, back, code_words, sf_word, a.et + (c0 - s0) * a.np + n, a.np);
     uint4 *dst = reinterpret_cast<uint4 *>(a.codes + n * (a.K / 2) + c0 / 2);
     dst[0] = make_uint4(code_words[0], code_words[1], code_words[2], code_words[3]);
     dst[1] = make_uint4(code_words[4], code_words[5], code_words[6], code_words[7]);

@@ -45,6 +45,21 @@ def test_gptq_matches_oracle(orc, fmt, had, N, K):
     assert_bytes_equal(s, orc.tc_scale_layout(osf), "scales")
 
 
+@pytest.mark.parametrize("had", [0, 16])
+@pytest.mark.parametrize("N,K", [(24, 128), (200, 320), (1, 64), (130, 512)])
+def test_gptq_mse_matches_oracle(orc, had, N, K):
+    w, u = _case(orc, N, K, had, 3 * N + K)
+    codes = torch.full((N, K // 2), 0xAA, dtype=torch.uint8, device=DEV)
+    scales = torch.full((fl.scale_bytes(N, K // 16),), 0xFF, dtype=torch.uint8, device=DEV)
+    c, s, g = fl.gptq_quantize(w.to(DEV), torch.from_numpy(u).to(DEV), "nvfp4", had, codes=codes, scales=scales,
+                               mse=True)
+    status_ok()
+    oc, osf, og = orc.gptq(w, u, "nvfp4", had, mse=True)
+    assert np.float32(g.item()).view(np.uint32) == np.float32(og).view(np.uint32)
+    assert_bytes_equal(c.cpu().numpy(), oc, "codes")
+    assert_bytes_equal(s.cpu().numpy(), orc.tc_scale_layout(osf), "scales")
+
+
 def test_gptq_static_scale(orc):
     N, K = 64, 256
     w, u = _case(orc, N, K, 16, 5)
