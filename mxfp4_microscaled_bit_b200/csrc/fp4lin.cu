@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "gemm_sm100.cuh"
 #include "gemm_sm100_2sm.cuh"
+#include "gemm_sm100_2sm_decode.cuh"
 #include "kv.cuh"
 #include "kv_attention.cuh"
 #include "gptq.cuh"
@@ -30,7 +31,7 @@ struct DeviceInfo {
     int status = FP4LIN_OK;
     int sms = 0;
     bool gemm_attr[7] = {false, false, false, false, false, false, false};
-    int pair_clusters[2] = {0, 0};  // resident clusters of the pair kernels (0: not yet queried)
+    int pair_clusters[4] = {0, 0, 0, 0};  // resident clusters of the pair kernels (0: not yet queried)
     bool attn_attr[KA_GMAX + 1] = {};  // dynamic shared memory raised for kv_attn_tc_kernel<G>
     bool gptq_attr = false;            // dynamic shared memory raised for gptq_update_kernel
 };
@@ -367,6 +368,119 @@ int launch_gemm_pair(DeviceInfo *dev, int slot, const uint8_t *a_codes, const ui
     return launch_status();
 }
 
+// The decode GEMM (M <= 16) on CTA pairs: 256 weight rows per pair, K split s ways over the
+// pairs, s chosen as plan_decode does but for pairs and only among splits whose partial sums
+// fit the caller's workspace.
+GemmPlan plan_decode_pair(int64_t M, int64_t N, int64_t K, int pairs, size_t ws_avail)
+{
+    GemmPlan p{};
+    p.swap = true;
+    p.bn = 16;
+    p.num_mt = (int)((N + 255) / 256);
+    p.num_nt = 1;
+    p.nk = (int)((K + 255) / 256);
+    p.ldw = (N + 3) / 4 * 4;
+    p.splits = 1;
+    p.kps = p.nk;
+    double best = 1e300;
+    for (int s = 1; s <= std::min(p.nk, 16); ++s) {
+        const int kps = (p.nk + s - 1) / s;
+        const int eff = (p.nk + kps - 1) / kps;
+        if (eff != s)
+            continue;
+        const size_t need = (size_t)s * (size_t)M * (size_t)p.ldw * sizeof(float);
+        if (s > 1 && need > ws_avail)
+            continue;
+        const int64_t waves = ((int64_t)p.num_mt * s + pairs - 1) / pairs;
+        double cost = (double)(waves * kps);
+        if (s > 1)
+            cost += 4.0 + 2.0 * s * (double)M * (double)p.ldw * 4.0 / (2.0 * pairs * 18432.0);
+        if (cost < best) {
+            best = cost;
+            p.splits = s;
+            p.kps = kps;
+        }
+    }
+    p.ws_bytes = p.splits > 1 ? (size_t)p.splits * (size_t)M * (size_t)p.ldw * sizeof(float) : 0;
+    return p;
+}
+
+// Whether the decode GEMM runs on CTA pairs (the default; FP4LIN_DECODE_KERNEL=single keeps
+// the one-CTA form).  Both give the same results.
+bool use_decode_pair()
+{
+    const char *e = getenv("FP4LIN_DECODE_KERNEL");
+    return !(e && strcmp(e, "single") == 0);
+}
+
+template <bool NV>
+int launch_decode_pair(DeviceInfo *dev, const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a,
+                       const uint8_t *w_codes, const uint8_t *w_scales, const float *g_w, void *y, int64_t M,
+                       int64_t N, int64_t K, int64_t ldy, void *workspace, size_t workspace_bytes, cudaStream_t st)
+{
+    using C = GemmDecodePairCfg<NV>;
+    const int slot = NV ? 2 : 3;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        if (dev->pair_clusters[slot] == 0) {
+            if (cudaFuncSetAttribute(fp4_gemm_decode_pair_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM_BYTES) != cudaSuccess)
+                return FP4LIN_ERR_CUDA;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3((unsigned)(dev->sms & ~1));
+            cfg.blockDim = dim3(C::THREADS);
+            cfg.dynamicSmemBytes = C::SMEM_BYTES;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, fp4_gemm_decode_pair_kernel<C>, &cfg) != cudaSuccess || n < 1)
+                return FP4LIN_ERR_CUDA;
+            dev->pair_clusters[slot] = n;
+        }
+    }
+    const int pairs = dev->pair_clusters[slot];
+    const GemmPlan pl = plan_decode_pair(M, N, K, pairs, workspace ? workspace_bytes : 0);
+    const int64_t sf_cols = NV ? K / 16 : K / 32;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB;
+    if (!make_code_map(&tmA, w_codes, N, K, 128) || !make_code_map(&tmB, a_codes, M, K, C::CN) ||
+        !make_scale_map(&tmSFA, w_scales, N, sf_cols, C::SF_BOX_ROWS) ||
+        !make_scale_map(&tmSFB, a_scales, M, sf_cols, C::SF_BOX_ROWS))
+        return FP4LIN_ERR_CUDA;
+    GemmDecodePairParams p{};
+    p.g_a = g_w;  // swapped slots: the MMA's A is the weights
+    p.g_w = g_a;
+    p.y = reinterpret_cast<__nv_bfloat16 *>(y);
+    p.ws = reinterpret_cast<float *>(workspace);
+    p.Nw = N;
+    p.Mact = M;
+    p.K = K;
+    p.ldy = ldy;
+    p.ldw = pl.ldw;
+    p.katoms = (sf_cols + 3) / 4;
+    p.katoms_act = p.katoms;
+    p.num_mt = pl.num_mt;
+    p.nk = pl.nk;
+    p.kps = pl.kps;
+    p.splits = pl.splits;
+    p.work = (int64_t)pl.num_mt * pl.splits;
+    const int64_t clusters = std::min<int64_t>(p.work, pairs);
+    fp4_gemm_decode_pair_kernel<C><<<(unsigned)(2 * clusters), C::THREADS, C::SMEM_BYTES, st>>>(tmA, tmB, tmSFA, tmSFB,
+                                                                                               p);
+    if (launch_status() != FP4LIN_OK)
+        return FP4LIN_ERR_CUDA;
+    if (pl.splits > 1) {
+        const int64_t items = M * ((N + 3) / 4);
+        const int rgrid = (int)std::min<int64_t>((items + 255) / 256, (int64_t)dev->sms * 8);
+        if (launch_pdl(splitk_reduce_kernel, rgrid, 256, 0, st, (const float *)workspace, pl.splits, M, N, pl.ldw,
+                       NV ? g_w : nullptr, NV ? g_a : nullptr, reinterpret_cast<__nv_bfloat16 *>(y), ldy,
+                       QuantOut{}) != cudaSuccess) {
+            cudaGetLastError();
+            return FP4LIN_ERR_CUDA;
+        }
+        if (launch_status() != FP4LIN_OK)
+            return FP4LIN_ERR_CUDA;
+    }
+    return FP4LIN_OK;
+}
+
 int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a, const uint8_t *w_codes,
                const uint8_t *w_scales, const float *g_w, void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
                void *workspace, size_t workspace_bytes, void *stream, const QuantOut &qo = QuantOut{},
@@ -400,6 +514,13 @@ int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const f
     }
     float *ws = reinterpret_cast<float *>(workspace);
     cudaStream_t s = as_stream(stream);
+    if (pl.swap && !quant && !w_tiled && use_decode_pair()) {  // CTA pairs: half the issue per weight row
+        if (nv)
+            return launch_decode_pair<true>(dev, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N, K, ldy,
+                                            workspace, workspace_bytes, s);
+        return launch_decode_pair<false>(dev, a_codes, a_scales, nullptr, w_codes, w_scales, nullptr, y, M, N, K, ldy,
+                                         workspace, workspace_bytes, s);
+    }
     if (pl.swap) {  // the weights take the MMA's M side: operands and shapes swap places
         if (nv)
             return launch_gemm_cfg<GemmCfg<16, true, true>>(dev, 4, pl, w_codes, w_scales, g_w, a_codes, a_scales,

@@ -87,3 +87,43 @@ def test_kernels_agree_bitwise(monkeypatch):
         status_ok()
     diff = (out["single"].view(torch.int16) != out["pair"].view(torch.int16)).sum().item()
     assert diff == 0, f"{diff} elements differ between the kernels"
+
+
+# ---------------------------------------------------------------- the decode GEMM on CTA pairs
+DECODE_CASES = [(1, 64, 64), (16, 256, 256), (5, 320, 1088), (16, 4096, 4096), (4, 14336, 4096), (16, 4096, 14336),
+                (9, 4224, 512)]
+
+
+@pytest.mark.parametrize("M,N,K", DECODE_CASES)
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_decode_pair_matches_single_and_oracle(orc, monkeypatch, M, N, K, fmt):
+    # the pair issues, per output element, the same K-ordered 64-deep MMAs as the one-CTA
+    # decode form (M = 256 instead of 128 on the weight side): the same bits, split or not
+    A = si.student_t_bf16(M + N, M, K)
+    W = si.normal_bf16(N + K, N, K, std=0.02)
+    out = {}
+    for kernel in ("single", "pair"):
+        monkeypatch.setenv("FP4LIN_DECODE_KERNEL", kernel)
+        for ws in ("auto", False):
+            kw = {} if ws == "auto" else {"workspace": ws}
+            if fmt == "nvfp4":
+                ca, sa, ga = fl.nvfp4_quantize(A.to(DEV), 16)
+                cw, sw, gw = fl.nvfp4_quantize(W.to(DEV), 16)
+                out[kernel, ws] = fl.nvfp4_gemm(ca, sa, ga, cw, sw, gw, **kw)
+            else:
+                ca, sa = fl.mxfp4_quantize(A.to(DEV), 32)
+                cw, sw = fl.mxfp4_quantize(W.to(DEV), 32)
+                out[kernel, ws] = fl.mxfp4_gemm(ca, sa, cw, sw, **kw)
+            status_ok()
+    for ws in ("auto", False):
+        assert torch.equal(out["pair", ws].view(torch.int16), out["single", ws].view(torch.int16)), ws
+    # and against the oracle's product (the unsplit pair output)
+    if fmt == "nvfp4":
+        oca, osa, oga = orc.nvfp4_quantize(A, 16)
+        ocw, osw, ogw = orc.nvfp4_quantize(W, 16)
+        yr, s = orc.gemm_abt(orc.dequant(oca, osa, "nvfp4", oga), orc.dequant(ocw, osw, "nvfp4", ogw))
+    else:
+        oca, osa = orc.mxfp4_quantize(A, 32)
+        ocw, osw = orc.mxfp4_quantize(W, 32)
+        yr, s = orc.gemm_abt(orc.dequant(oca, osa, "mxfp4"), orc.dequant(ocw, osw, "mxfp4"))
+    check_gemm_values(orc, out["pair", False].float().cpu().numpy(), yr, s, f"decode pair {fmt} {M}x{N}x{K}")
