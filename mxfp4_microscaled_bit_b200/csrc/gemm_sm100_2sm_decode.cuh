@@ -7,6 +7,10 @@
 // M = 256: the leader issues one scale-A copy (each CTA copies its own 128 rows), one scale-B
 // copy and one MMA for 256 weight rows -- half the instructions per weight row.
 //
+// Measured, it is slower than the one-CTA form (16x14336x4096: 16.5 against 15.0 us): the
+// pair's instructions and its completions on the leader's barriers cost more each, so it runs
+// only when FP4LIN_DECODE_KERNEL=pair asks for it.  Its results are the same, bit for bit.
+//
 // Roles (320 threads per CTA, both CTAs of the pair):
 //   warp 0 lane 0   producer: TMA loads of this CTA's 128 weight rows, its 8 of the 16
 //                   activation rows, its weight scale atoms and all activation scale atoms
