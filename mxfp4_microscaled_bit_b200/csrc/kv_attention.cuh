@@ -112,21 +112,6 @@ __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi)
     return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
 }
 
-// Halves (lo of x, lo of y) or (hi of x, hi of y) of two f16x2 words.
-__device__ __forceinline__ uint32_t prmt_lo(uint32_t x, uint32_t y)
-{
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(x), "r"(y));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t prmt_hi(uint32_t x, uint32_t y)
-{
-    uint32_t r;
-    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(x), "r"(y));
-    return r;
-}
-
 // Tensor-core form of the split kernel (same workspace output).  The CTA first stages its
 // chunk in shared memory: the K and V code rows (contiguous per kv head) by one bulk async
 // copy each, the scale rows by cooperative 8-byte loads, so every byte of the chunk is in
@@ -139,8 +124,9 @@ __device__ __forceinline__ uint32_t prmt_hi(uint32_t x, uint32_t y)
 // Pass 2: o += p v by mma_16816x, A = the weights of 16 positions for 8 heads in rows 0..7
 // and the f16 rounding of what the f16 weights leave out in rows 8..15 (so p keeps ~22
 // bits and one MMA accumulates both), B = V with the output dimensions permuted so that a
-// lane needs 16 contiguous dimensions (8 code bytes, one scale) of each of its 4 rows; prmt
-// pairs two rows' values into one fragment register.
+// lane needs 16 contiguous dimensions (8 code bytes, one scale) of each of its 4 rows; the
+// code nibbles of two rows are interleaved before the conversion, so each converted pair is
+// already a fragment register (one row per half).
 template <int G>
 __global__ void __launch_bounds__(KA_THREADS, 4) kv_attn_tc_kernel(KvAttnShape a)
 {
@@ -305,26 +291,44 @@ __global__ void __launch_bounds__(KA_THREADS, 4) kv_attn_tc_kernel(KvAttnShape a
         const float2 b01 = half2_to_float2(ah0), b23 = half2_to_float2(ah2);
         const uint32_t al0 = f16x2_bits(__fsub_rn(p4[0], b01.x), __fsub_rn(p4[1], b01.y));
         const uint32_t al2 = f16x2_bits(__fsub_rn(p4[2], b23.x), __fsub_rn(p4[3], b23.y));
-        uint32_t hv[4][8];  // rows rp[0..3], dimensions 16gq + 2k, 2k + 1
+        // rows rp[0..3]: their code words (dimensions 16gq .. 16gq + 15) and scale bytes
+        uint2 c[4];
+        uint32_t sfb[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            uint2 c = make_uint2(0u, 0u);
-            uint32_t sfb = 0u;
+            c[e] = make_uint2(0u, 0u);
+            sfb[e] = 0u;
             if (rp[e] < n) {
-                c = *reinterpret_cast<const uint2 *>(s_vc + rp[e] * (KA_D / 2) + 8 * gq);
-                sfb = s_vs[rp[e] * 8 + gq];
+                c[e] = *reinterpret_cast<const uint2 *>(s_vc + rp[e] * (KA_D / 2) + 8 * gq);
+                sfb[e] = s_vs[rp[e] * 8 + gq];
             }
-            const uint32_t s2u = kv_scale_pair(sfb * 0x101u);
-            kv_fp8_word(c.x, s2u, hv[e]);
-            kv_fp8_word(c.y, s2u, hv[e] + 4);
+        }
+        // B fragments: for dimension 16gq + u, (row 2t, row 2t+1) in bv[0][u], (row 2t+8, row 2t+9) in
+        // bv[1][u].  The two rows' code nibbles are interleaved first -- byte j of `ev` holds dimension
+        // 2j of both rows, of `od` dimension 2j+1 -- so each conversion yields such a pair directly,
+        // scaled by the two rows' own scales (low half: the first row).
+        uint32_t bv[2][16];
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+            const uint32_t s2u = kv_scale_pair(sfb[2 * pr] | (sfb[2 * pr + 1] << 8));
+#pragma unroll
+            for (int hw = 0; hw < 2; ++hw) {  // dimensions 0..7, then 8..15
+                const uint32_t x0 = hw ? c[2 * pr].y : c[2 * pr].x, x1 = hw ? c[2 * pr + 1].y : c[2 * pr + 1].x;
+                const uint32_t ev = (x0 & 0x0F0F0F0Fu) | ((x1 & 0x0F0F0F0Fu) << 4);
+                const uint32_t od = ((x0 >> 4) & 0x0F0F0F0Fu) | (x1 & 0xF0F0F0F0u);
+                uint32_t he[4], ho[4];
+                kv_fp8_word(ev, s2u, he);
+                kv_fp8_word(od, s2u, ho);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    bv[pr][8 * hw + 2 * j] = he[j];
+                    bv[pr][8 * hw + 2 * j + 1] = ho[j];
+                }
+            }
         }
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const int k = u >> 1;
-            const uint32_t b0 = (u & 1) ? prmt_hi(hv[0][k], hv[1][k]) : prmt_lo(hv[0][k], hv[1][k]);
-            const uint32_t b1 = (u & 1) ? prmt_hi(hv[2][k], hv[3][k]) : prmt_lo(hv[2][k], hv[3][k]);
-            mma_16816x(o[u], ah0, al0, ah2, al2, b0, b1);
-        }
+        for (int u = 0; u < 16; ++u)
+            mma_16816x(o[u], ah0, al0, ah2, al2, bv[0][u], bv[1][u]);
     }
     __syncthreads();  // every thread has read the weights: reuse s_buf for the warps' outputs
     if (gq < G)
