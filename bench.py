@@ -521,6 +521,26 @@ def main():
         w.mxfp4_layer()
     mx_ms = time_loop(w.mxfp4_layer, 20, stream) / 20
 
+    # ---- the MXFP4 comparison on the prefill shape: relative Frobenius error of each format's layer
+    #      output (with and without rotation) against the float64 product of the unquantised
+    #      operands, on the first 128 activation rows (every weight row)
+    def rel_frobenius():
+        rows = 128
+        exact = w.A[:rows].double() @ w.W_bf16.double().T
+        out = {}
+        for name, fmt, had in (("nvfp4_h16", "nvfp4", 16), ("nvfp4", "nvfp4", 0), ("mxfp4_h32", "mxfp4", 32),
+                               ("mxfp4", "mxfp4", 0)):
+            wq = w.w if (fmt, had) == ("nvfp4", 16) else (w.w_mx if (fmt, had) == ("mxfp4", 32)
+                                                          else fl.prepare_weight(w.W_bf16, fmt, had))
+            lin = fl.nvfp4_linear if fmt == "nvfp4" else fl.mxfp4_linear
+            y = lin(w.A, wq)[:rows].double()
+            out[name] = float((y - exact).norm() / exact.norm())
+            del wq
+        return out
+
+    c3_err = rel_frobenius()
+    assert fl.device_status() == 0
+
     # ---- the output handed to a next NVFP4 layer: GEMM then quantiser vs the fused epilogue
     w.chained_setup()
     for _ in range(3):
@@ -687,6 +707,11 @@ def main():
                     "kv_load_gbs": rooflines["kv_load_fp8"]["achieved"],
                     "kv_store_us": st_ms * 1e3,
                     "mxfp4_layer_tflops": flops / (mx_ms * 1e-3) / 1e12,
+                    "mxfp4_vs_nvfp4": {"layer_tflops": {"nvfp4_h16": layer_tf, "mxfp4_h32": flops / (mx_ms * 1e-3) / 1e12},
+                                       "rel_frobenius_error": c3_err,
+                                       "note": "prefill shape; errors of the layer output on activation rows "
+                                               "0..127 against the float64 product of the unquantised bf16 "
+                                               "operands"},
                     "bf16_matmul_context": {"ms": bf16_ms, "tflops": flops / (bf16_ms * 1e-3) / 1e12,
                                             "layer_speedup": bf16_ms / layer_ms, "gemm_speedup": bf16_ms / gemm_ms,
                                             "note": "torch.matmul (cuBLAS) bf16 on the unquantised prefill "
