@@ -184,6 +184,25 @@ int fp4lin_convert_selftest(const float *in, uint8_t *e2m1, uint8_t *e4m3, int64
                             void *stream);
 
 /*
+ * Diagnostic of the device-side wait limit.  One CTA runs two waits on
+ * shared-memory barriers through the same bounded-wait routine the GEMM
+ * pipelines use: wait 1 with a limit of limit_ns nanoseconds, wait 0 with the
+ * library's 1 s limit but giving up as soon as another wait of the CTA has
+ * expired (the GEMM's abort rule).
+ *   arrive = 1: each barrier is arrived on first; both waits succeed and the
+ *               device status stays FP4LIN_OK.
+ *   arrive = 0: nothing arrives.  Wait 1 expires after limit_ns and records
+ *               FP4LIN_ERR_TIMEOUT in the device status; wait 0 then gives
+ *               up.  The kernel returns normally: the context stays usable.
+ * result: device, 4 x uint64, 8-byte aligned, written by the kernel:
+ *   result[0], result[1] = 1 if wait 0 / wait 1 saw its barrier complete;
+ *   result[2], result[3] = nanoseconds wait 0 / wait 1 took (global timer).
+ * limit_ns in [1000, 100000000] (1 us .. 100 ms), else
+ * FP4LIN_ERR_INVALID_ARGUMENT, as for arrive not 0 or 1 or result NULL.
+ */
+int fp4lin_wait_selftest(uint64_t limit_ns, int arrive, uint64_t *result, void *stream);
+
+/*
  * nvfp4_quantize with the tensor scale computed (compute_global_scale = 1),
  * for callers that cannot allocate device memory: plug-ins whose host
  * framework owns the whole device memory pool and forbids raw cudaMalloc, or

@@ -10,7 +10,7 @@ Entry points (same names as the C ABI in include/fp4lin.h):
   nvfp4_quantize, nvfp4_gemm, mxfp4_quantize, mxfp4_gemm,
   kv_nvfp4_store, kv_nvfp4_load_fp8
 plus helpers: scale_bytes, gemm_workspace_bytes, device_status,
-convert_selftest, prepare_weight, nvfp4_linear, mxfp4_linear.
+convert_selftest, wait_selftest, prepare_weight, nvfp4_linear, mxfp4_linear.
 """
 from __future__ import annotations
 
@@ -26,7 +26,7 @@ from . import build as _build
 __all__ = [
     "Fp4LinError", "lib", "nvfp4_quantize", "nvfp4_gemm", "mxfp4_quantize", "mxfp4_gemm",
     "kv_nvfp4_store", "kv_nvfp4_load_fp8", "scale_bytes", "gemm_workspace_bytes",
-    "device_status", "convert_selftest", "QuantizedWeight", "prepare_weight", "nvfp4_linear",
+    "device_status", "convert_selftest", "wait_selftest", "QuantizedWeight", "prepare_weight", "nvfp4_linear",
     "mxfp4_linear", "nvfp4_linear_decode", "tile_weights", "nvfp4_gemm_tiled", "gptq_quantize", "gptq_hessian_factor", "prepare_weight_gptq",
     "EXPORTS",
 ]
@@ -48,6 +48,7 @@ EXPORTS = {
     "kv_nvfp4_load_fp8": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _int, _int, _i64, _int, _vp]),
     "fp4lin_device_status": (_int, [_vp]),
     "fp4lin_convert_selftest": (_int, [_vp, _vp, _vp, _i64, _vp]),
+    "fp4lin_wait_selftest": (_int, [ctypes.c_uint64, _int, _vp, _vp]),
     "nvfp4_quantize_noalloc": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_mse": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_quantize_nearest": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _vp, _vp]),
@@ -341,6 +342,18 @@ def convert_selftest(x: torch.Tensor, stream=None):
     e4 = torch.empty(n, dtype=torch.uint8, device=x.device)
     _check("fp4lin_convert_selftest", lib().fp4lin_convert_selftest(_ptr(x), _ptr(e2), _ptr(e4), n, _stream(stream)))
     return e2, e4
+
+
+def wait_selftest(limit_ns: int, arrive: bool, device=None, stream=None) -> torch.Tensor:
+    """Run the device-side bounded wait (diagnostic): two barrier waits in one CTA, the
+    second limited to limit_ns.  Without `arrive` nothing completes them, so the second
+    expires and records TIMEOUT in the device status, and the first gives up after it.
+    Returns the int64 tensor [done0, done1, ns0, ns1] on the device."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    r = torch.full((4,), -1, dtype=torch.int64, device=dev)
+    _check("fp4lin_wait_selftest", lib().fp4lin_wait_selftest(int(limit_ns), 1 if arrive else 0, _ptr(r),
+                                                               _stream(stream)))
+    return r
 
 
 # ------------------------------------------------------------------ layer helpers

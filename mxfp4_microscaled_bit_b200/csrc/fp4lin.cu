@@ -1120,6 +1120,21 @@ int fp4lin_device_status(void *stream)
     return (int)v;
 }
 
+int fp4lin_wait_selftest(uint64_t limit_ns, int arrive, uint64_t *result, void *stream)
+{
+    if (!result || limit_ns < 1000ull || limit_ns > 100000000ull || (arrive != 0 && arrive != 1))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (!aligned(result, 8))
+        return FP4LIN_ERR_MISALIGNED;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    wait_selftest_kernel<<<1, 64, 0, as_stream(stream)>>>((unsigned long long)limit_ns, arrive,
+                                                          reinterpret_cast<unsigned long long *>(result));
+    return launch_status();
+}
+
 int fp4lin_convert_selftest(const float *in, uint8_t *e2m1, uint8_t *e4m3, int64_t n, void *stream)
 {
     if (!in || !e2m1 || !e4m3 || n < 1)

@@ -62,9 +62,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Wait for the phase of `bar` with parity `parity`.  Returns false if it gave
-// up: after WAIT_LIMIT_NS (records a timeout and raises *abort), or, when
+// up: after limit_ns (records a timeout and raises *abort), or, when
 // honor_abort, as soon as another role has raised *abort.
-__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort, bool honor_abort)
+__device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort, bool honor_abort,
+                                          unsigned long long limit_ns = WAIT_LIMIT_NS)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -75,7 +76,7 @@ __device__ __noinline__ bool wait_bounded(uint64_t *bar, uint32_t parity, volati
         if ((it & 7u) == 0u) {
             if (honor_abort && *abort)
                 return false;
-            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 report_error(FP4LIN_ERR_TIMEOUT);
                 *abort = 1;
                 return false;
@@ -113,6 +114,37 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     if (lane == 0)
         ok = wait_bar(bar, parity, abort) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Diagnostic of the expiry path of wait_bounded, the wait every pipeline role
+// uses.  Two single-arrival barriers; lane 0 of warp w waits on barrier w.
+// Warp 1 waits with limit_ns, warp 0 with the kernel limit but honouring the
+// CTA abort flag, as the GEMM's roles do.  With arrive != 0 each barrier gets
+// its arrival first and both waits succeed.  Without it nothing ever arrives:
+// warp 1's wait expires (records FP4LIN_ERR_TIMEOUT, raises the flag) and
+// warp 0's gives up on seeing the flag.  Every loop ends by the clock.
+// result[w] = 1 if warp w's wait saw the phase complete, else 0;
+// result[2 + w] = nanoseconds warp w spent waiting.
+__global__ void __launch_bounds__(64, 1)
+    wait_selftest_kernel(unsigned long long limit_ns, int arrive, unsigned long long *result)
+{
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        abort_flag = 0;
+    }
+    __syncthreads();
+    if (lane != 0)
+        return;
+    if (arrive)
+        mbar_arrive(&bars[warp]);
+    const unsigned long long t0 = globaltimer_ns();
+    const bool ok = wait_bounded(&bars[warp], 0, &abort_flag, warp == 0, warp == 1 ? limit_ns : WAIT_LIMIT_NS);
+    result[2 + warp] = globaltimer_ns() - t0;
+    result[warp] = ok ? 1ull : 0ull;
 }
 
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y)

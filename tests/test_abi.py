@@ -23,7 +23,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported():
     names = header_functions()
-    assert len(names) == 28, names
+    assert len(names) == 29, names
     L = fl.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -106,6 +106,12 @@ def test_kv_argument_checks():
     assert L.kv_nvfp4_load_fp8(P, P, P, 9, P, P, 2, 2, 8, 128, None) == INVALID  # L > Lcap
     assert L.kv_nvfp4_load_fp8(P, P, P, 8, P + 1, P, 2, 2, 8, 128, None) == MISALIGNED
     assert L.fp4lin_convert_selftest(P, P, P, 0, None) == INVALID
+    # the wait diagnostic: limit outside [1 us, 100 ms], arrive not 0/1, no result buffer
+    assert L.fp4lin_wait_selftest(999, 0, P, None) == INVALID
+    assert L.fp4lin_wait_selftest(100000001, 0, P, None) == INVALID
+    assert L.fp4lin_wait_selftest(10000, 2, P, None) == INVALID
+    assert L.fp4lin_wait_selftest(10000, 0, None, None) == INVALID
+    assert L.fp4lin_wait_selftest(10000, 0, P + 4, None) == MISALIGNED
 
 
 def d(M=16, K=128, ldx=128, had=0, dyn=0, ga=P, x=P, y=P, N=64, ldy=64, ws=P, wsb=8192):
