@@ -129,13 +129,45 @@ __device__ __forceinline__ float e4m3_value(uint32_t b)
 // NVFP4 block scale from the block maximum and the FP32 tensor scale g:
 // t = (amax/6)/g, sf = E4M3(t), d = dec(sf)*g; returns sf and sets rcp = 1/d
 // (0 when d = 0).  The one arithmetic every NVFP4 encoder in this library uses.
+// 1/d for scale byte sf, d = dec(sf)*g; 0 when d is not positive.
+__device__ __forceinline__ float nvfp4_block_rcp(uint32_t sf, float g)
+{
+    const float d = __fmul_rn(e4m3_value(sf), g);
+    return d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+}
+
 __device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float g, float &rcp)
 {
     const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
     const uint32_t sf = cvt_e4m3(t);
-    const float d = __fmul_rn(e4m3_value(sf), g);
-    rcp = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+    rcp = nvfp4_block_rcp(sf, g);
     return sf;
+}
+
+// The scale byte of nvfp4_block_scale, E4M3((amax/6)/g), from one product where that gives
+// the same byte.  c6 = nvfp4_fast_c6(g) approximates 1/(6g) within 2 rounding errors, so
+// ta = amax*c6 is within 3 relative rounding errors of amax/(6g) and the two-division
+// quotient within 2: the two differ by less than 6 units in the last place of ta's binade.
+// Rounding to E4M3 keeps mantissa bits 22..20 and rounds on bits 19..0; its midpoints are
+// bits 19..0 = 0x80000.  So where ta is in the normal E4M3 range (>= 2^-6), finite, and more
+// than 32 units from such a midpoint, both round to the same byte (near a power of two,
+// where the two may sit in adjacent binades, both round to that power).  Everything else
+// (midpoint neighbourhoods, the subnormal range, non-finite values, g outside the range
+// nvfp4_fast_c6 accepts) takes the two divisions.
+__device__ __forceinline__ float nvfp4_fast_c6(float g)
+{
+    return (g >= 0x1p-100f && g <= 0x1p+100f) ? __fdiv_rn(1.0f, __fmul_rn(6.0f, g)) : __int_as_float(0x7fc00000);
+}
+
+__device__ __forceinline__ uint32_t nvfp4_scale_code_fast(float amax, float g, float c6)
+{
+    const float ta = __fmul_rn(amax, c6);
+    const int off = (int)(__float_as_uint(ta) & 0xFFFFFu) - 0x80000;
+    if (ta >= 0x1p-6f && ta <= 0x1.fffffep+127f && (off > 32 || off < -32))
+        return cvt_e4m3(ta);
+    if (amax == 0.0f && c6 > 0.0f)  // (0/6)/g = 0 for a finite positive g
+        return 0u;
+    return cvt_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
 }
 
 // ------------------------------------------------------------------ packed binary32 pairs

@@ -213,17 +213,21 @@ __global__ void __launch_bounds__(QTHREADS) nvfp4_amax_kernel(QuantShape q, floa
 // Pass 2: quantise.  DYNAMIC: g = max(partials) / (6*448) (1 if not > 0),
 // written to g_io by CTA (0,0); otherwise g is read from g_io.
 // Per block: t = (amax/6)/g, sf = E4M3(t), d = dec(sf)*g, r = d > 0 ? 1/d : 0,
-// codes = E2M1(x'*r).
+// codes = E2M1(x'*r).  sf comes from nvfp4_scale_code_fast (one product, the two divisions
+// only where that product could round differently) and r from a per-CTA table over the 256
+// scale bytes: the same bytes and codes as nvfp4_block_scale.
 template <bool HAD, bool DYNAMIC>
-__global__ void __launch_bounds__(QTHREADS)
+__global__ void __launch_bounds__(QTHREADS, 4)  // four CTAs per SM: at most 64 registers
     nvfp4_quant_kernel(QuantShape q, float *g_io, const float *partials, int n_partials)
 {
     __shared__ float s_g;
     __shared__ float red[QWARPS];
+    __shared__ float s_rcp[256];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t c = (int64_t)blockIdx.x * 32 + lane;
     const bool col_ok = c < q.blocks_per_row;
     const int64_t r0 = (int64_t)blockIdx.y * QROWS + warp;
+    static_assert(QROWS == 32 && QWARPS == 8, "a CTA's rows are one 32-row group of the scale layout");
     // issue the loads first; the tensor-scale reduction overlaps them
     uint32_t raw[QUNROLL][8];
 #pragma unroll
@@ -263,6 +267,13 @@ __global__ void __launch_bounds__(QTHREADS)
     }
     __syncthreads();
     const float g = s_g;
+    // 1/(dec(sf)*g) for every scale byte, once per CTA instead of once per block
+    static_assert(QTHREADS == 256, "one table entry per thread");
+    s_rcp[threadIdx.x] = nvfp4_block_rcp(threadIdx.x, g);
+    __syncthreads();
+    const float c6 = nvfp4_fast_c6(g);
+    // the QUNROLL rows of a thread share their 32-row group: scale bytes 128 apart
+    const int64_t sbase = tc_offset(r0, c, q.katoms);
 #pragma unroll
     for (int u = 0; u < QUNROLL; ++u) {
         const int64_t r = r0 + QWARPS * u;
@@ -270,11 +281,10 @@ __global__ void __launch_bounds__(QTHREADS)
             continue;
         float v[16];
         nvfp4_block_values<HAD>(raw[u], v);
-        float rcp;
-        const uint32_t sf = nvfp4_block_scale(abs_max<16>(v), g, rcp);
-        scale_packed<16>(v, rcp);
+        const uint32_t sf = nvfp4_scale_code_fast(abs_max<16>(v), g, c6);
+        scale_packed<16>(v, s_rcp[sf]);
         *reinterpret_cast<uint2 *>(q.codes + r * (q.cols / 2) + c * 8) = make_uint2(pack_e2m1x8(v), pack_e2m1x8(v + 8));
-        q.scales[tc_offset(r, c, q.katoms)] = (uint8_t)sf;
+        q.scales[sbase + 128 * u] = (uint8_t)sf;
     }
 }
 

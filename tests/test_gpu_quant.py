@@ -118,6 +118,27 @@ def test_nvfp4_static_scale(orc, g):
     check_nvfp4(orc, si.student_t_bf16(78, 64, 256), 16, g)
 
 
+@pytest.mark.parametrize("k", [0, 3, 7])
+def test_nvfp4_block_scale_near_e4m3_midpoints(orc, k):
+    # Block j has maximum 1536 * 2^-j (exact in bf16), so (amax/6)/g = 256/g * 2^-j exactly
+    # (barring underflow).  g is chosen so that 256/g lands within +-40 binary32 units of the
+    # E4M3 rounding midpoint (1 + (2k+1)/16) * 2^8; every block then carries the same offset
+    # from a midpoint into its own binade, through the normal, subnormal and zero range of
+    # E4M3.  Both sides of each midpoint must round as the two-division definition does.
+    mid = 1.0 + (2 * k + 1) / 16.0
+    rows, cols = 8, 64  # 32 blocks
+    j = np.arange(32, dtype=np.float64)
+    amax = 1536.0 * 2.0 ** -j
+    frac = np.array([1.0] + [((-1) ** i) * i / 16.0 for i in range(1, 16)])
+    x = (amax[:, None] * frac[None, :]).astype(np.float32).reshape(rows, cols)
+    xb = si.to_bf16(x)
+    assert torch.equal(xb.float().abs().reshape(32, 16).amax(1), torch.from_numpy(amax.astype(np.float32)))
+    for d in range(-40, 41):
+        g = float(np.float32(1.0 / (mid * (1.0 + d * 2.0 ** -23))))
+        check_nvfp4(orc, xb, 0, g)
+    status_ok()
+
+
 def test_nvfp4_zero_and_tiny_tensors(orc):
     check_nvfp4(orc, torch.zeros(3, 64, dtype=torch.bfloat16))
     tiny = si.normal_bf16(9, 5, 128, std=1e-30)
