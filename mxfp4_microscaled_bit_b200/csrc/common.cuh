@@ -127,8 +127,9 @@ __device__ __forceinline__ float e4m3_value(uint32_t b)
 }
 
 // NVFP4 block scale from the block maximum and the FP32 tensor scale g:
-// t = (amax/6)/g, sf = E4M3(t), d = dec(sf)*g; returns sf and sets rcp = 1/d
-// (0 when d = 0).  The one arithmetic every NVFP4 encoder in this library uses.
+// t = (amax/6)/g, sf = E4M3(t), d = dec(sf)*g, rcp = 1/d (0 when d is not positive).
+// The one arithmetic every NVFP4 encoder in this library uses (nvfp4_block_scale below).
+
 // 1/d for scale byte sf, d = dec(sf)*g; 0 when d is not positive.
 __device__ __forceinline__ float nvfp4_block_rcp(uint32_t sf, float g)
 {
@@ -136,13 +137,6 @@ __device__ __forceinline__ float nvfp4_block_rcp(uint32_t sf, float g)
     return d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
 }
 
-__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float g, float &rcp)
-{
-    const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
-    const uint32_t sf = cvt_e4m3(t);
-    rcp = nvfp4_block_rcp(sf, g);
-    return sf;
-}
 
 // The scale byte of nvfp4_block_scale, E4M3((amax/6)/g), from one product where that gives
 // the same byte.  c6 = nvfp4_fast_c6(g) approximates 1/(6g) within 2 rounding errors, so
@@ -168,6 +162,15 @@ __device__ __forceinline__ uint32_t nvfp4_scale_code_fast(float amax, float g, f
     if (amax == 0.0f && c6 > 0.0f)  // (0/6)/g = 0 for a finite positive g
         return 0u;
     return cvt_e4m3(__fdiv_rn(__fdiv_rn(amax, 6.0f), g));
+}
+
+// NVFP4 block scale byte and rcp as defined above.  Callers that encode many blocks with one
+// g get nvfp4_fast_c6(g) computed once (the compiler hoists it out of their loops).
+__device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float g, float &rcp)
+{
+    const uint32_t sf = nvfp4_scale_code_fast(amax, g, nvfp4_fast_c6(g));
+    rcp = nvfp4_block_rcp(sf, g);
+    return sf;
 }
 
 // ------------------------------------------------------------------ packed binary32 pairs
