@@ -3,9 +3,11 @@ inputs once, then calls one entry point `--iters` times.  Inputs are larger than
 the 126 MB L2 but hold at most a few GB on the device.
 
   python -m mxfp4_microscaled_bit_b200.profile_cases --case gemm_prefill --iters 3
+  python -m mxfp4_microscaled_bit_b200.profile_cases --case quant_prefill --iters 30 --time-cold write
 cases: gemm_prefill (8192 x 14336 x 4096 NVFP4, 16-wide rotation), gemm_mxfp4,
 gemm_decode (16 x 14336 x 4096), quant_prefill (8192 x 4096 rotated, dynamic
-scale), kv_load (8 x 8 x 32768 x 128 cache to FP8), kv_store, kv_attention (decode
+scale; _static: the tensor scale given; _static_h0: given, no rotation),
+kv_load (8 x 8 x 32768 x 128 cache to FP8), kv_store, kv_attention (decode
 attention over the same 8 x 8 caches, G = 4), quant_mse (the 14336 x 4096 weight,
 MSE-optimal scales), gemm_quant (the prefill GEMM with its output NVFP4-encoded),
 linear_decode (16 x 14336 x 4096 with the activation quantiser inside the GEMM),
@@ -29,9 +31,13 @@ import synthetic_inputs as si  # noqa: E402
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--case", required=True,
-                    choices=["gemm_prefill", "gemm_mxfp4", "gemm_decode", "quant_prefill", "kv_load", "kv_store",
-                             "kv_attention", "quant_mse", "gemm_quant", "linear_decode", "gptq"])
+                    choices=["gemm_prefill", "gemm_mxfp4", "gemm_decode", "quant_prefill", "quant_prefill_static",
+                             "quant_prefill_static_h0", "kv_load", "kv_store", "kv_attention", "quant_mse",
+                             "gemm_quant", "linear_decode", "gptq"])
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--time-cold", choices=["write", "read"], default=None,
+                    help="time each call with CUDA events after flushing the L2 by writing (or reading) "
+                         "512 MiB; print the mean")
     a = ap.parse_args()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
@@ -53,10 +59,15 @@ def main():
     elif a.case == "quant_mse":
         W = si.prefill_W().to(dev)
         fn = lambda: fl.nvfp4_quantize(W, 16, mse=True)  # noqa: E731
-    elif a.case in ("gemm_prefill", "gemm_mxfp4", "quant_prefill", "gemm_quant"):
+    elif a.case in ("gemm_prefill", "gemm_mxfp4", "quant_prefill", "quant_prefill_static",
+                    "quant_prefill_static_h0", "gemm_quant"):
         A = si.prefill_A().to(dev)
         if a.case == "quant_prefill":
             fn = lambda: fl.nvfp4_quantize(A, 16)  # noqa: E731
+        elif a.case.startswith("quant_prefill_static"):
+            had = 0 if a.case.endswith("h0") else 16
+            c, s, g = fl.nvfp4_quantize(A, had)  # the tensor scale, then reused as a static one
+            fn = lambda: fl.nvfp4_quantize(A, had, g, codes=c, scales=s)  # noqa: E731
         elif a.case == "gemm_quant":
             w = fl.prepare_weight(si.prefill_W().to(dev), "nvfp4", 16)
             ca, sa, ga = fl.nvfp4_quantize(A, 16)
@@ -107,6 +118,24 @@ def main():
             new = xd[:, :, :1].contiguous()
             pos = torch.full((B,), L - 1, dtype=torch.int32, device=dev)
             fn = lambda: fl.kv_nvfp4_store(new, pos, g, codes, scales)  # noqa: E731
+    if a.time_cold:
+        flush = torch.empty(512 * 2**20, dtype=torch.uint8, device=dev)
+        fn()
+        total = 0.0
+        for _ in range(a.iters):
+            if a.time_cold == "write":
+                flush.zero_()
+            else:
+                flush.view(torch.int64).sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            total += e0.elapsed_time(e1)
+        assert fl.device_status() == 0
+        print(f"{a.case}: {total / a.iters * 1e3:.1f} us per call (mean of {a.iters}, L2 flushed by {a.time_cold})")
+        return
     for _ in range(a.iters):
         fn()
     torch.cuda.synchronize()
