@@ -113,8 +113,11 @@ __device__ __forceinline__ uint4 kv_block_fp8(uint2 c, uint32_t sf)
 
 // Wide path: a thread takes 8 consecutive blocks -- 64 code bytes (two 256-bit
 // loads), 8 scale bytes (one 64-bit load), 128 FP8 bytes out (four 256-bit
-// stores) -- and keeps two such groups in flight.  Taken when the slice's
-// block count and every base are aligned for it (see kv_load_fp8_wide_ok).
+// stores) -- and keeps KV_WIDE_INFLIGHT such groups in flight.  Taken when the
+// slice's block count and every base are aligned for it (see kv_load_fp8_wide_ok).
+// Four groups (120 registers, two CTAs per SM) keep more loads in flight per SM
+// than two (73 registers, three CTAs) or one (32 registers, eight CTAs).
+constexpr int KV_WIDE_INFLIGHT = 4;
 __device__ __forceinline__ void kv_load_group8(const uint8_t *codes, const uint8_t *scales, uint8_t *out, int64_t grp,
                                                uint32_t *c, uint2 &sf)
 {
@@ -134,17 +137,17 @@ __global__ void __launch_bounds__(KV_THREADS) kv_load_fp8_wide_kernel(KvLoadShap
     const uint8_t *scales = s.scales + bh * s.Lcap * s.bpr;
     uint8_t *out = s.out + bh * nblk * 16;
     const int64_t stride = (int64_t)gridDim.x * KV_THREADS;
-    for (int64_t g0 = (int64_t)blockIdx.x * KV_THREADS + threadIdx.x; g0 < ngrp; g0 += 2 * stride) {
-        uint32_t c[2][16];
-        uint2 sf[2];
+    for (int64_t g0 = (int64_t)blockIdx.x * KV_THREADS + threadIdx.x; g0 < ngrp; g0 += KV_WIDE_INFLIGHT * stride) {
+        uint32_t c[KV_WIDE_INFLIGHT][16];
+        uint2 sf[KV_WIDE_INFLIGHT];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < KV_WIDE_INFLIGHT; ++u) {
             const int64_t grp = g0 + u * stride;
             if (grp < ngrp)
                 kv_load_group8(codes, scales, out, grp, c[u], sf[u]);
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < KV_WIDE_INFLIGHT; ++u) {
             const int64_t grp = g0 + u * stride;
             if (grp >= ngrp)
                 continue;
