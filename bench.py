@@ -45,8 +45,8 @@ FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP
 # DRAM bytes (read + write) per step for a kernel, from one ncu capture of the current build
 # (summarised under profiles/); None where no capture covers the kernel as it stands.
 NCU_TRAFFIC = {
-    "gemm": 290.8e6,          # the 8192x14336x4096 prefill GEMM, one launch
-    "kv_load_fp8": None,      # kernel changed since its last capture
+    "gemm": 288.5e6,          # the 8192x14336x4096 prefill GEMM, one launch
+    "kv_load_fp8": 5.882e9,   # 367.6 MB per 8x8x32768x128 cache, x 8 (units) x 2 (K, V)
     "quantize": None,         # the capture covers the quantise pass only, not the amax pass
     "kv_store": None,
 }
