@@ -172,3 +172,26 @@ def test_nvfp4_beats_mxfp4_error(orc):
         errs[name] = np.linalg.norm(y - exact) / np.linalg.norm(exact)
     print("relative Frobenius errors", errs)
     assert errs["nv"] < errs["mx"] and errs["nv_h"] < errs["mx_h"]
+
+
+def test_binding_refuses_undersized_buffers():
+    # a caller-supplied buffer smaller than what the call writes raises before any launch
+    x = si.normal_bf16(3, 32, 128).to(DEV)
+    codes = torch.full((32, 64), 0xAA, dtype=torch.uint8, device=DEV)
+    small = torch.full((100,), 0xAA, dtype=torch.uint8, device=DEV)  # the layout needs 512 bytes
+    with pytest.raises(ValueError, match="scales holds 100 bytes"):
+        fl.nvfp4_quantize(x, 0, codes=codes, scales=small)
+    torch.cuda.synchronize()
+    assert bool((codes == 0xAA).all()) and bool((small == 0xAA).all())
+    c, s, g = fl.nvfp4_quantize(x)
+    y_small = torch.full((16, 32), 7.0, dtype=torch.bfloat16, device=DEV)  # 32 rows are written
+    with pytest.raises(ValueError, match="out holds"):
+        fl.nvfp4_gemm(c, s, g, c, s, g, out=y_small)
+    torch.cuda.synchronize()
+    assert bool((y_small == 7.0).all())
+    with pytest.raises(ValueError, match="out_scale must be contiguous|out holds"):
+        kc = torch.zeros(1, 1, 8, 64, dtype=torch.uint8, device=DEV)
+        ks = torch.full((1, 1, 8, 8), 0x38, dtype=torch.uint8, device=DEV)
+        fl.kv_nvfp4_load_fp8(kc, ks, torch.ones(1, device=DEV), 8, out=torch.empty(1, 1, 4, 128, dtype=torch.uint8,
+                                                                                     device=DEV))
+    status_ok()
