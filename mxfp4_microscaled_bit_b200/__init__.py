@@ -8,9 +8,17 @@ raises.
 
 Entry points (same names as the C ABI in include/fp4lin.h):
   nvfp4_quantize, nvfp4_gemm, mxfp4_quantize, mxfp4_gemm,
-  kv_nvfp4_store, kv_nvfp4_load_fp8
-plus helpers: scale_bytes, gemm_workspace_bytes, device_status,
-convert_selftest, wait_selftest, prepare_weight, nvfp4_linear, mxfp4_linear.
+  kv_nvfp4_store, kv_nvfp4_load_fp8, kv_nvfp4_attention, nvfp4_gemm_quant,
+  nvfp4_linear_decode, nvfp4_gemm_tiled, gptq_quantize
+plus helpers: scale_bytes, gemm_workspace_bytes, tile_weights, device_status,
+convert_selftest, wait_selftest, prepare_weight, prepare_weight_gptq,
+gptq_hessian_factor, nvfp4_linear, mxfp4_linear.
+
+Errors: a caller-supplied tensor of the wrong dtype raises TypeError; one in host
+memory, on another device, in a layout the call cannot take, or smaller than the
+call reads or writes raises ValueError -- all before anything is launched.  A
+status other than OK from the library raises Fp4LinError.  Timeouts and
+out-of-range KV positions found on the device are reported by device_status().
 """
 from __future__ import annotations
 
