@@ -46,10 +46,8 @@ __global__ void __launch_bounds__(KV_THREADS) kv_store_kernel(KvStoreShape s)
         for (int j = 0; j < 8; ++j)
             amax = fmaxf(amax, fabsf(v[j]));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        const float t = __fdiv_rn(__fdiv_rn(amax, 6.0f), g);
-        const uint32_t sf = cvt_e4m3(t);
-        const float d = __fmul_rn(e4m3_value(sf), g);
-        const float rcp = d > 0.0f ? __fdiv_rn(1.0f, d) : 0.0f;
+        float rcp;
+        const uint32_t sf = nvfp4_block_scale(amax, g, rcp);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             v[j] = __fmul_rn(v[j], rcp);
