@@ -15,9 +15,11 @@ CPU oracle baseline are reported beside it.  Usage:
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-With N > 1 it is launched by torch.distributed.run, one rank per GPU; each rank
-runs the same workload on its own GPU (replicas: the path has no exchange
-step), and times are the maximum over ranks.
+With N > 1 it runs one rank per GPU under torch.distributed.run: either the
+caller launches it so (WORLD_SIZE must then equal N), or, when WORLD_SIZE is
+unset, bench.py re-launches itself that way.  Each rank runs the same workload on
+its own GPU (replicas: the path has no exchange step), and times are the maximum
+over ranks.
 """
 from __future__ import annotations
 
@@ -50,6 +52,12 @@ NCU_TRAFFIC = {
     "quantize": None,         # the capture covers the quantise pass only, not the amax pass
     "kv_store": None,
 }
+# How each traffic figure was taken, where it is not a full-size launch.
+NCU_TRAFFIC_NOTE = {
+    "kv_load_fp8": "lower bound: DRAM bytes of an 8x8x32768x128 capture scaled x16 by the units processed; up to "
+                   "~50 MB of that launch's writes were still in L2 when it ended, so the scaled figure reads "
+                   "below the 6.711 GB algorithmic minimum",
+}
 METRIC = "NVFP4 GEMM TFLOP/s (% dense FP4 peak); quantize/KV GB/s (% of HBM)"
 
 
@@ -78,6 +86,34 @@ def max_over_ranks(x: float, device="cpu") -> float:
 def barrier():
     if torch.distributed.is_available() and torch.distributed.is_initialized():
         torch.distributed.barrier()
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def relaunch(n: int, argv: list[str]) -> int:
+    """Run this script again under torch.distributed.run with n ranks on this node (127.0.0.1);
+    rank 0's JSON line reaches our stdout.  Returns the launcher's exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def launch_check() -> int:
+    """The launch alone, on CPU: join the process group over gloo, take the maximum of the rank
+    numbers over all ranks, rank 0 prints it."""
+    rank, _, ws = dist_init("gloo")
+    m = max_over_ranks(float(rank))
+    barrier()
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "n_gpus": ws, "max_rank": m}), flush=True)
+    if torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+    return 0
 
 
 def load_peaks():
@@ -239,11 +275,17 @@ class Workload:
 
     LAUNCHES_PER_STEP = 7  # amax + quantise + GEMM + 2 KV stores + 2 KV loads
 
-    def mxfp4_layer(self):
+    def mxfp4_layer(self, ev=None):
         fl = self.fl
+        if ev is not None:
+            ev[0].record()
         fl.mxfp4_quantize(self.A, 32, codes=self.a_codes, scales=self.a_scales_mx)
+        if ev is not None:
+            ev[1].record()
         fl.mxfp4_gemm(self.a_codes, self.a_scales_mx, self.w_mx.codes, self.w_mx.scales, out=self.y,
                       workspace=False)
+        if ev is not None:
+            ev[2].record()
 
     # the layer's output as the next layer's NVFP4 input (static tensor scale, 16-wide rotation)
     def chained_setup(self):
@@ -468,8 +510,21 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-rows", type=int, default=1024)
+    ap.add_argument("--launch-check", action="store_true",
+                    help="only start the N ranks, join them over gloo and report (no GPU work)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.gpus < 1:
+        print(f"bench.py: --gpus must be >= 1, not {args.gpus}", file=sys.stderr)
+        return 2
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return relaunch(args.gpus, sys.argv[1:])
+    if dist_env()[2] != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={dist_env()[2]}: launch one rank per GPU",
+              file=sys.stderr)
+        return 2
+    if args.launch_check:
+        return launch_check()
 
     if args.impl == "reference":
         return reference_arm(args)
@@ -516,10 +571,16 @@ def main():
     layer_ms_max = max_over_ranks(layer_ms, dev)
     gemm_ms_max = max_over_ranks(gemm_ms, dev)
 
-    # ---- MXFP4 variant of the same layer (reported, not part of the step)
+    # ---- MXFP4 variant of the same layer (reported, not part of the step): quantise + GEMM, the
+    #      GEMM's own time from events around it
     for _ in range(3):
         w.mxfp4_layer()
-    mx_ms = time_loop(w.mxfp4_layer, 20, stream) / 20
+    mx_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(20)]
+    for e in mx_ev:
+        w.mxfp4_layer(e)
+    torch.cuda.synchronize()
+    mx_ms = float(np.mean([e[0].elapsed_time(e[2]) for e in mx_ev]))
+    mx_gemm_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in mx_ev]))
 
     # ---- the MXFP4 comparison on the prefill shape: relative Frobenius error of each format's layer
     #      output (with and without rotation) against the float64 product of the unquantised
@@ -664,23 +725,41 @@ def main():
                 "traffic": None, "algorithmic_bytes": bytes_, "ms": ms}
 
     gemm_tf = flops / (gemm_ms * 1e-3) / 1e12
+    # the FP4 tensor pipe's own rate at the sampled clock: one 128x256x64 block-scaled MMA per SM
+    # every 128 cycles (measured with a stream of MMAs and no other work), 148 SMs
+    clock_fp4 = 148 * (2 * 128 * 256 * 64 / 128) * float(clk.get("sm_mhz") or 1965.0) * 1e6 / 1e12
+    mx_gemm_tf = flops / (mx_gemm_ms * 1e-3) / 1e12
     rooflines = {
-        "gemm": {"bound": "tensor", "achieved": gemm_tf, "peak": sustained_fp4, "unit": "TFLOP/s",
-                 "frac": gemm_tf / sustained_fp4, "traffic": None, "ms": gemm_ms,
-                 "peak_basis": f"{peak_src} bf16 sustained x {FP4_PER_BF16:g} (dense FP4 : BF16)",
-                 "frac_of_burst_fp4": gemm_tf / burst_fp4, "frac_of_datasheet_9pf": gemm_tf / 9000.0},
+        "gemm": {"bound": "tensor", "achieved": gemm_tf, "peak": burst_fp4, "unit": "TFLOP/s",
+                 "frac": gemm_tf / burst_fp4, "traffic": None, "ms": gemm_ms,
+                 "peak_basis": f"{peak_src} bf16 burst x {FP4_PER_BF16:g} (dense FP4 : BF16); the step's GEMMs "
+                               f"run in a short region at full clock",
+                 "frac_of_sustained_fp4": gemm_tf / sustained_fp4, "frac_of_clock_fp4": gemm_tf / clock_fp4,
+                 "clock_fp4_tflops": clock_fp4, "frac_of_datasheet_9pf": gemm_tf / 9000.0},
+        "mxfp4_gemm": {"bound": "tensor", "achieved": mx_gemm_tf, "peak": burst_fp4, "unit": "TFLOP/s",
+                       "frac": mx_gemm_tf / burst_fp4, "traffic": None, "ms": mx_gemm_ms,
+                       "frac_of_clock_fp4": mx_gemm_tf / clock_fp4},
         "kv_load_fp8": hbm_roof(w.kv_load_bytes(), ld_ms),
         "quantize": hbm_roof(w.quant_bytes(), q_ms),
         "kv_store": hbm_roof(w.kv_store_bytes(), st_ms),
     }
     for k, r in rooflines.items():
         r["traffic"] = NCU_TRAFFIC.get(k)
+        if k in NCU_TRAFFIC_NOTE:
+            r["traffic_note"] = NCU_TRAFFIC_NOTE[k]
     rooflines["quantize"]["note"] = "2.5625 B/element (one read of A); the dynamic tensor scale reads A twice"
     rooflines["kv_load_fp8"]["frac_of_8tbs"] = rooflines["kv_load_fp8"]["achieved"] / 8000.0
     shares = {"quantize": q_ms, "gemm": gemm_ms, "kv_store": st_ms, "kv_load_fp8": ld_ms}
     dominant = max(shares, key=shares.get)
     roof = dict(rooflines[dominant])
     roof["kernel"] = dominant
+    # every timed kernel's roofline in brief, beside the dominant one's
+    roof["kernels"] = {k: {"achieved": r["achieved"], "peak": r["peak"], "unit": r["unit"], "frac": r["frac"],
+                           "ms": r["ms"]} for k, r in rooflines.items()}
+    roof["kernels"]["gemm"]["frac_of_clock_fp4"] = gemm_tf / clock_fp4
+    roof["kernels"]["mxfp4_gemm"]["frac_of_clock_fp4"] = mx_gemm_tf / clock_fp4
+    roof["kernels"]["mxfp4_gemm"]["layer_tflops"] = flops / (mx_ms * 1e-3) / 1e12
+    roof["kernels"]["mxfp4_gemm"]["rel_frobenius_error"] = c3_err
 
     layer_tf = ws * flops / (layer_ms_max * 1e-3) / 1e12
     line = {
@@ -702,7 +781,7 @@ def main():
         "step_ms": {"quantize": q_ms, "gemm": gemm_ms, "kv_store": st_ms, "kv_load_fp8": ld_ms,
                     "layer": layer_ms, "share": {k: v / sum(shares.values()) for k, v in shares.items()}},
         "metrics": {"layer_tflops": layer_tf, "gemm_tflops": gemm_tf,
-                    "gemm_frac_dense_fp4": gemm_tf / sustained_fp4,
+                    "gemm_frac_dense_fp4": gemm_tf / burst_fp4,
                     "quantize_gbs": rooflines["quantize"]["achieved"],
                     "kv_load_gbs": rooflines["kv_load_fp8"]["achieved"],
                     "kv_store_us": st_ms * 1e3,

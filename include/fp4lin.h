@@ -15,7 +15,8 @@
  *     the rotation folded into the weights: the MR-GPTQ abstract
  *     (hyper.ai/de/papers/2509.23202), "Abstract".
  *   - KV cache written in NVFP4, dequantised to FP8 before attention: the
- *     NVFP4 KV-cache story (hyper.ai/de/stories/...).
+ *     NVFP4 KV-cache story (hyper.ai/de/stories/e1307393ec176dd2b0276468adeec3f9,
+ *     one untitled paragraph).
  *
  * Conventions for every entry point:
  *   - All data pointers are DEVICE pointers on the current CUDA device; the
@@ -58,7 +59,9 @@ enum fp4lin_status {
     FP4LIN_ERR_TIMEOUT = 5,          /* a device-side wait gave up (reported by fp4lin_device_status) */
     FP4LIN_ERR_DEVICE = 6,           /* the current device is not compute capability 10.0 (B200) */
     FP4LIN_ERR_WORKSPACE = 7,        /* workspace null or smaller than required */
-    FP4LIN_ERR_OUT_OF_RANGE = 8      /* a KV position outside [0, Lcap) (reported by fp4lin_device_status) */
+    FP4LIN_ERR_OUT_OF_RANGE = 8,     /* a KV position outside [0, Lcap) (reported by fp4lin_device_status) */
+    FP4LIN_ERR_NUMERIC = 9           /* a factorisation met a pivot that is not positive and finite
+                                        (reported by fp4lin_device_status) */
 };
 
 /* Library version, MAJOR*10000 + MINOR*100 + PATCH. */
@@ -79,6 +82,11 @@ size_t fp4lin_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
  * NVFP4 quantisation of a bf16 matrix, optionally rotated.
+ * Defined by: "FP4 auf Blackwell: Was NVFP4 fuer lokale KI wirklich aendert", section
+ * "Was NVFP4 von frueheren 4-Bit-Formaten unterscheidet" (E2M1 elements, E4M3 block scale per 16
+ * values, one FP32 scale per tensor); "FP8, NVFP4 czy AWQ?", section "Czym roznia sie FP8, NVFP4, MXFP4 i AWQ?",
+ * NVFP4 bullet (16-element blocks, FP8 E4M3 scale); the rotation: the MR-GPTQ abstract (hyper.ai/de/papers/2509.23202), "Abstract"
+ * (blockwise Hadamard transforms, activations rotated online).
  *
  *   x       [rows, cols] bf16, row stride ld_x elements.
  *   hadamard 0 (none) or 16: rotate every 16-value block along the row by
@@ -104,6 +112,12 @@ int nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
 
 /*
  * y[M, N] = A[M, K] * W[N, K]^T for NVFP4 operands, FP32 accumulation on the
+ * tensor cores.  Defined by: "FP4 auf Blackwell: Was NVFP4 fuer lokale KI wirklich aendert", section
+ * "Was NVFP4 von frueheren 4-Bit-Formaten unterscheidet"
+ * (Blackwell's 5th-generation tensor cores apply the two-level scaling in
+ * hardware); "FP8, NVFP4 czy AWQ?", section "Dlaczego W8A8 i W4A16 to nie to
+ * samo?" (W4A4: weights and activations both 4-bit, the product on low-precision
+ * tensor cores).  Result:
  * tensor cores, y = bf16_round(g_a * g_w * acc).
  *   a_codes [M, K/2], a_scales tensor-core layout of [M, K/16];
  *   w_codes [N, K/2], w_scales tensor-core layout of [N, K/16];
@@ -118,7 +132,12 @@ int nvfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales, const float *g_a
                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * MXFP4 quantisation: 32-value blocks, E8M0 scale byte = clamp(X + 127, 0,
+ * MXFP4 quantisation.  Defined by: "FP4 auf Blackwell: Was NVFP4 fuer lokale KI wirklich aendert", section
+ * "Was NVFP4 von frueheren 4-Bit-Formaten unterscheidet"
+ * (MXFP4: 32-value blocks scaled by powers of two); "FP8, NVFP4 czy AWQ?", section "Czym roznia sie FP8, NVFP4, MXFP4 i AWQ?",
+ * MXFP4 bullet (the OCP Microscaling standard's E8M0 block scale); the 32-wide
+ * rotation: the MR-GPTQ abstract (hyper.ai/de/papers/2509.23202), "Abstract".
+ * 32-value blocks, E8M0 scale byte = clamp(X + 127, 0,
  * 254) with X = floor(log2 amax) - 2, codes = E2M1 of x' * 2^-X.
  *   hadamard 0 or 32 (rotate each 32-value block by H_32 / sqrt(32)).
  *   codes [rows, cols/2]; scales tensor-core layout of [rows, cols/32].
@@ -128,7 +147,11 @@ int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                    int hadamard, uint8_t *codes, uint8_t *scales, void *stream);
 
 /* y = A * W^T for MXFP4 operands (E8M0 scales, no tensor scale); otherwise
- * as nvfp4_gemm. */
+ * as nvfp4_gemm.
+ * Defined by: "FP4 auf Blackwell: Was NVFP4 fuer lokale KI wirklich aendert", section
+ * "Was NVFP4 von frueheren 4-Bit-Formaten unterscheidet"
+ * (MXFP4 blocks of 32 with power-of-two scales, multiplied on the block-scaled
+ * tensor cores); "FP8, NVFP4 czy AWQ?", section "Czym roznia sie FP8, NVFP4, MXFP4 i AWQ?", MXFP4 bullet. */
 int mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales,
                const uint8_t *w_codes, const uint8_t *w_scales,
                void *y, int64_t M, int64_t N, int64_t K, int64_t ldy,
@@ -136,6 +159,9 @@ int mxfp4_gemm(const uint8_t *a_codes, const uint8_t *a_scales,
 
 /*
  * Append T new K (or V) rows per (batch, head) to an NVFP4 cache.
+ * Defined by: the NVFP4 KV-cache story (hyper.ai/de/stories/e1307393ec176dd2b0276468adeec3f9,
+ * one untitled paragraph), its statement that new K/V vectors are written to the
+ * cache in NVFP4 and the KV tensors are dequantised to FP8 before attention.
  *   kv_new       bf16 [B, H, T, D] contiguous.
  *   pos          device int32 [B]: row t of batch b goes to position pos[b] + t.
  *   g            device float, the static FP32 tensor scale (> 0).
@@ -153,7 +179,10 @@ int kv_nvfp4_store(const void *kv_new, const int32_t *pos, const float *g,
 
 /*
  * Dequantise the first L positions of every (batch, head) of an NVFP4 cache
- * to FP8 E4M3 for attention:
+ * to FP8 E4M3 for attention.
+ * Defined by: the NVFP4 KV-cache story (hyper.ai/de/stories/e1307393ec176dd2b0276468adeec3f9,
+ * one untitled paragraph), its statement that new K/V vectors are written to the
+ * cache in NVFP4 and the KV tensors are dequantised to FP8 before attention.
  *   out_fp8[b,h,l,d] = E4M3_rne(e2m1(code) * dec(sf) / 8), out_scale = 8 * g,
  * so that value = fp8 * out_scale.  The product is exact, so the E4M3
  * rounding is the only rounding.
@@ -217,7 +246,10 @@ int fp4lin_wait_selftest(uint64_t limit_ns, int arrive, uint64_t *result, void *
  * The call allocates nothing (no cudaMalloc, cudaFree or allocating library
  * routine).  The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture.  All calls on a device share the array and it keeps the last
+ * stream capture.  The cached address belongs to the device's primary context
+ * as it was at that first call: after cudaDeviceReset on a device, do not call
+ * this entry point on that device again in the same process (the address
+ * would be stale); nvfp4_quantize with a caller workspace is unaffected.  All calls on a device share the array and it keeps the last
  * call's contents (nothing in it has to start at zero: each call overwrites
  * every partial it reads), so calls that overlap on the GPU -- on different
  * streams without ordering -- race and must be avoided.
@@ -360,6 +392,36 @@ int nvfp4_linear_decode(const void *x, int64_t M, int64_t K, int64_t ld_x, int h
  * gives FP4LIN_ERR_WORKSPACE.  Time grows as N K^2 (binary32 multiply-adds).
  */
 size_t gptq_workspace_bytes(int64_t N, int64_t K);
+/*
+ * GPTQ's input from calibration activations: the factor u that the MR-GPTQ
+ * entry points above take.  Defined by: the MR-GPTQ abstract
+ * (hyper.ai/de/papers/2509.23202), "Abstract" -- MR-GPTQ is a variant of the
+ * classic GPTQ algorithm with blockwise Hadamard transforms, so its Hessian
+ * is that of the rotated layer inputs.  In binary64:
+ *   x' = x blockdiag(H_b / sqrt b)   (b = hadamard: 16, 32, or 0 = none)
+ *   H  = x'^T x' + damp * mean(diag(x'^T x')) * I
+ *   u  = the upper triangular factor with positive diagonal, H^-1 = u^T u,
+ *        rounded to float (entries below the diagonal written 0).
+ * u is found without forming H^-1: with P the reversal of the K indices,
+ * P H P = L L^T (blocked Cholesky, 64 x 64 blocks) and u = P L^-1 P.
+ *   x: double [T, K], row stride ld_x >= K (8-byte aligned), the calibration
+ *      activations (T tokens), unrotated;
+ *   damp >= 0 (GPTQ's usual choice is 0.01);
+ *   u: float [K, K], row stride ld_u >= K, 4-byte aligned;
+ *   workspace: gptq_hessian_workspace_bytes(T, K) bytes, 16-byte aligned:
+ *      8 * (T K + 2 K^2 + 128 K) bytes (the rotated activations, the
+ *      Hessian's factor and its inverse, and 64-row blocks of products).
+ * T >= 1; K a multiple of 64.  If H is not positive definite (a pivot not
+ * positive and finite, e.g. all-zero or non-finite x with damp = 0),
+ * FP4LIN_ERR_NUMERIC is recorded in the device status word (see
+ * fp4lin_device_status) and u is not meaningful.  Other errors as
+ * nvfp4_quantize; a workspace below the size gives FP4LIN_ERR_WORKSPACE.
+ * Time grows as T K^2 + K^3 (binary64 multiply-adds).
+ */
+size_t gptq_hessian_workspace_bytes(int64_t T, int64_t K);
+int gptq_hessian_factor(const double *x, int64_t T, int64_t K, int64_t ld_x, int hadamard,
+                        double damp, float *u, int64_t ld_u,
+                        void *workspace, size_t workspace_bytes, void *stream);
 int nvfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int hadamard,
                         const float *u, int64_t ld_u, int compute_global_scale, float *g,
                         uint8_t *codes, uint8_t *scales,

@@ -40,7 +40,7 @@ __all__ = [
 ]
 
 STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA",
-          5: "TIMEOUT", 6: "DEVICE", 7: "WORKSPACE", 8: "OUT_OF_RANGE"}
+          5: "TIMEOUT", 6: "DEVICE", 7: "WORKSPACE", 8: "OUT_OF_RANGE", 9: "NUMERIC"}
 
 _i64, _sz, _vp, _int = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_int
 EXPORTS = {
@@ -77,6 +77,8 @@ EXPORTS = {
     "mxfp4_gptq_quantize": (_int, [_vp, _i64, _i64, _i64, _int, _vp, _i64, _vp, _vp, _vp, _sz, _vp]),
     "nvfp4_linear_decode": (_int, [_vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _vp, _sz,
                                    _vp]),
+    "gptq_hessian_workspace_bytes": (_sz, [_i64, _i64]),
+    "gptq_hessian_factor": (_int, [_vp, _i64, _i64, _i64, _int, ctypes.c_double, _vp, _i64, _vp, _sz, _vp]),
 }
 
 _lock = threading.Lock()
@@ -542,24 +544,28 @@ def prepare_weight(w: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0, tiled
 
 
 # ------------------------------------------------------------------ MR-GPTQ (offline weights)
-def gptq_hessian_factor(x: torch.Tensor, hadamard: int = 0, damp: float = 0.01) -> torch.Tensor:
-    """Preparation of GPTQ's input, plain dense linear algebra in float64 on x's device: the
-    calibration activations x [T, K] rotated blockwise by H_b / sqrt(b) (b = hadamard), the
-    damped Hessian H = x'^T x' + damp * mean(diag) I, and the upper factor U with
-    H^-1 = U^T U.  Returns U as float32 [K, K]."""
-    xd = x.to(torch.float64)
-    T, K = xd.shape
-    if hadamard:
-        h = torch.ones(1, 1, dtype=torch.float64, device=x.device)
-        while h.shape[0] < hadamard:
-            h = torch.cat([torch.cat([h, h], 1), torch.cat([h, -h], 1)], 0)
-        xd = (xd.reshape(T, K // hadamard, hadamard) @ (h / hadamard ** 0.5).T).reshape(T, K)
-    H = xd.T @ xd
-    H.diagonal().add_(damp * H.diagonal().mean())
-    L = torch.linalg.cholesky(H)
-    Hinv = torch.cholesky_inverse(L)
-    U = torch.linalg.cholesky((Hinv + Hinv.T) / 2, upper=True)
-    return U.to(torch.float32).contiguous()
+def gptq_hessian_factor(x: torch.Tensor, hadamard: int = 0, damp: float = 0.01, *, out=None, workspace=None,
+                        stream=None) -> torch.Tensor:
+    """GPTQ's input from calibration activations x [T, K] (float64, on the current device): the
+    library's gptq_hessian_factor -- x rotated blockwise by H_b / sqrt(b) (b = hadamard), the damped
+    Hessian H = x'^T x' + damp * mean(diag) I, and the upper factor U with H^-1 = U^T U, in
+    binary64.  Returns U as float32 [K, K] (out, if given).  A Hessian that is not positive
+    definite is reported by device_status() as NUMERIC (9)."""
+    fn = "gptq_hessian_factor"
+    _arg(fn, "x", x, torch.float64, rows=True)
+    T, K = x.shape
+    dev = x.device
+    if out is None:
+        out = torch.empty(K, K, dtype=torch.float32, device=dev)
+    else:
+        _arg(fn, "out", out, _F32, _rows_span(out, K, K), rows=True)
+    if workspace is None:
+        workspace = torch.empty(max(16, int(lib().gptq_hessian_workspace_bytes(T, K))), dtype=torch.uint8,
+                                device=dev)
+    wsb = _ws_arg(fn, workspace)
+    _check(fn, lib().gptq_hessian_factor(_ptr(x), T, K, x.stride(0), hadamard, float(damp), _ptr(out), out.stride(0),
+                                         _ptr(workspace), wsb, _stream(stream)))
+    return out
 
 
 def gptq_quantize(w: torch.Tensor, u: torch.Tensor, fmt: str = "nvfp4", hadamard: int = 0, g=None, *,

@@ -17,6 +17,7 @@
 #include "kv.cuh"
 #include "kv_attention.cuh"
 #include "gptq.cuh"
+#include "hessian.cuh"
 #include "quantize.cuh"
 #include "scale_search.cuh"
 
@@ -1448,6 +1449,84 @@ int mxfp4_gptq_quantize(const void *w, int64_t N, int64_t K, int64_t ld_w, int h
 {
     return gptq_entry(false, w, N, K, ld_w, hadamard, u, ld_u, 0, nullptr, codes, scales, workspace,
                       workspace_bytes, stream);
+}
+
+// Workspace of gptq_hessian_factor: the rotated, column-reversed activations [T, K], the
+// reversed Hessian and its factor [K, K], the factor's inverse [K, K], the inverses of its
+// 64 x 64 diagonal blocks [K / 64][64][64] and one 64 x K block row of products (all binary64).
+size_t gptq_hessian_workspace_bytes(int64_t T, int64_t K)
+{
+    if (T < 1 || K < 1 || K % HB != 0)
+        return 0;
+    return (size_t)(T * K + 2 * K * K + 2 * (int64_t)HB * K) * sizeof(double);
+}
+
+int gptq_hessian_factor(const double *x, int64_t T, int64_t K, int64_t ld_x, int hadamard, double damp, float *u,
+                        int64_t ld_u, void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!x || !u || !workspace)
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (T < 1 || K < 1 || ld_x < K || ld_u < K || (hadamard != 0 && hadamard != 16 && hadamard != 32) ||
+        !(damp >= 0.0) || !(damp < 1e300))
+        return FP4LIN_ERR_INVALID_ARGUMENT;
+    if (K % HB != 0 || K > (int64_t)1 << 20 || T > ((int64_t)1 << 40) / K)
+        return FP4LIN_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(x, 8) || !aligned(u, 4) || !aligned(workspace, 16))
+        return FP4LIN_ERR_MISALIGNED;
+    if (workspace_bytes < gptq_hessian_workspace_bytes(T, K))
+        return FP4LIN_ERR_WORKSPACE;
+    DeviceInfo *dev = nullptr;
+    int st = current_device(&dev);
+    if (st != FP4LIN_OK)
+        return st;
+    cudaStream_t s = as_stream(stream);
+    double *xr = reinterpret_cast<double *>(workspace);
+    double *A = xr + T * K;                // P H P, then its Cholesky factor Lr (lower triangle)
+    double *X = A + K * K;                 // Lr^-1
+    double *dinv = X + K * K;              // inverses of Lr's diagonal blocks
+    double *Tb = dinv + (int64_t)HB * K;   // one 64 x K block row of products
+    const int nblk = (int)(K / HB);
+    auto grid_for = [&](int64_t items) {
+        return (unsigned)std::max<int64_t>(1, std::min<int64_t>((items + 255) / 256, (int64_t)dev->sms * 8));
+    };
+    // 1. rotation, columns reversed
+    if (hadamard == 16)
+        hess_rotate_kernel<16><<<grid_for(T * (K / 16)), 256, 0, s>>>(x, T, K, ld_x, xr);
+    else if (hadamard == 32)
+        hess_rotate_kernel<32><<<grid_for(T * (K / 32)), 256, 0, s>>>(x, T, K, ld_x, xr);
+    else
+        hess_rotate_kernel<1><<<grid_for(T * K), 256, 0, s>>>(x, T, K, ld_x, xr);
+    // 2. the Gram product's lower triangle: A(m, n) = sum_t xr[t][m] xr[t][n]
+    {
+        DgemmArgs g{xr, xr, A, K, K, T, 1, K, 1, K, K, 0, 0, 0, 1.0, 0.0};
+        dgemm_kernel<false, false, true><<<dim3(nblk, nblk, 1), 256, 0, s>>>(g);
+    }
+    // 3. damping
+    hess_damp_kernel<<<1, 256, 0, s>>>(A, K, damp);
+    // 4. blocked Cholesky, right-looking
+    for (int kb = 0; kb < nblk; ++kb) {
+        chol_diag_kernel<<<1, 256, 0, s>>>(A, K, kb, dinv);
+        const int rem = nblk - kb - 1;
+        if (rem == 0)
+            break;
+        chol_panel_kernel<<<rem, 256, 0, s>>>(A, K, kb, dinv);
+        double *pan = A + (int64_t)(kb + 1) * HB * K + (int64_t)kb * HB;
+        double *trail = A + (int64_t)(kb + 1) * HB * K + (int64_t)(kb + 1) * HB;
+        DgemmArgs g{pan, pan, trail, (int64_t)rem * HB, (int64_t)rem * HB, HB, K, 1, K, 1, K, 0, 0, 0, -1.0, 1.0};
+        dgemm_kernel<true, true, true><<<dim3(rem, rem, 1), 256, 0, s>>>(g);
+    }
+    // 5. X = Lr^-1, one block row at a time: X[i, :i] = -D_i^-1 (Lr[i, :i] X[:i, :i])
+    hess_inv_init_kernel<<<grid_for(K * K), 256, 0, s>>>(X, K, dinv);
+    for (int i = 1; i < nblk; ++i) {
+        const int64_t w = (int64_t)i * HB;
+        DgemmArgs g1{A + w * K, X, Tb, HB, w, w, K, 1, 1, K, K, 0, 0, 0, 1.0, 0.0};
+        dgemm_kernel<true, false, false><<<dim3(i, 1, 1), 256, 0, s>>>(g1);
+        DgemmArgs g2{dinv + (int64_t)i * HB * HB, Tb, X + w * K, HB, w, HB, HB, 1, 1, K, K, 0, 0, 0, -1.0, 0.0};
+        dgemm_kernel<true, false, false><<<dim3(i, 1, 1), 256, 0, s>>>(g2);
+    }
+    // 6. U = P X P, upper triangle
+    hess_out_kernel<<<grid_for(K * K), 256, 0, s>>>(X, K, u, ld_u);
+    return cudaGetLastError() == cudaSuccess ? FP4LIN_OK : FP4LIN_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -1,7 +1,9 @@
 // kv.cuh -- NVFP4 KV cache: quantise appended K/V rows into the cache, and
-// dequantise the cache to FP8 E4M3 for attention (the NVFP4 KV-cache story,
-// hyper.ai/de/stories/...: new K/V vectors are written in NVFP4, the KV
-// tensors are dequantised to FP8 before the attention computation).
+// dequantise the cache to FP8 E4M3 for attention.  Source: the NVFP4 KV-cache
+// story (hyper.ai/de/stories/e1307393ec176dd2b0276468adeec3f9), a single
+// untitled paragraph; the passage used is its statement that new K/V vectors
+// are written to the cache in NVFP4 while the KV tensors are dequantised to
+// FP8 before the attention computation.
 #pragma once
 
 #include "common.cuh"

@@ -2,8 +2,8 @@
 inputs once, then calls one entry point `--iters` times.  Inputs are larger than
 the 126 MB L2 but hold at most a few GB on the device.
 
-  python -m mxfp4_microscaled_bit_b200.profile_cases --case gemm_prefill --iters 3
-  python -m mxfp4_microscaled_bit_b200.profile_cases --case quant_prefill --iters 30 --time-cold write
+  python profile_cases.py --case gemm_prefill --iters 3
+  python profile_cases.py --case quant_prefill --iters 30 --time-cold write
 cases: gemm_prefill (8192 x 14336 x 4096 NVFP4, 16-wide rotation), gemm_mxfp4,
 gemm_decode (16 x 14336 x 4096), quant_prefill (8192 x 4096 rotated, dynamic
 scale; _static: the tensor scale given; _static_h0: given, no rotation),
@@ -22,7 +22,7 @@ import sys
 import numpy as np
 import torch
 
-sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 
 import mxfp4_microscaled_bit_b200 as fl  # noqa: E402
 import synthetic_inputs as si  # noqa: E402

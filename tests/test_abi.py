@@ -23,7 +23,7 @@ def header_functions():
 
 def test_every_declared_symbol_is_exported():
     names = header_functions()
-    assert len(names) == 29, names
+    assert len(names) == 31, names
     L = fl.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -138,6 +138,30 @@ def test_gptq_argument_checks():
     assert q(wsp=None) == INVALID
     assert L.mxfp4_gptq_quantize(P, 64, 128, 128, 16, P, 128, P, P, P, ws, None) == INVALID  # 32 or 0
     assert L.mxfp4_gptq_quantize(P, 64, 96, 96, 32, P, 96, P, P, P, ws, None) == SHAPE
+
+
+def test_hessian_factor_argument_checks():
+    L = fl.lib()
+    ws = L.gptq_hessian_workspace_bytes(200, 128)
+    assert ws == 8 * (200 * 128 + 2 * 128 * 128 + 128 * 128)
+    assert L.gptq_hessian_workspace_bytes(200, 96) == 0  # K not a multiple of 64
+
+    def h(x=P, T=200, K=128, ldx=128, had=16, damp=0.01, u=P, ldu=128, wsp=P, wsb=ws):
+        return L.gptq_hessian_factor(x, T, K, ldx, had, damp, u, ldu, wsp, wsb, None)
+
+    assert h(x=None) == INVALID
+    assert h(u=None) == INVALID
+    assert h(wsp=None) == INVALID
+    assert h(T=0) == INVALID
+    assert h(ldx=127) == INVALID
+    assert h(ldu=64) == INVALID
+    assert h(had=8) == INVALID
+    assert h(damp=-0.5) == INVALID
+    assert h(damp=float("nan")) == INVALID
+    assert h(K=96, ldx=96, ldu=96, wsb=10 ** 9) == SHAPE
+    assert h(x=P + 4) == MISALIGNED
+    assert h(u=P + 2) == MISALIGNED
+    assert h(wsb=ws - 1) == WORKSPACE
 
 
 def test_tiled_weight_checks():

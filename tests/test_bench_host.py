@@ -63,3 +63,27 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch):
     class A:
         steps, warmup = 1, 0
     assert bench.reference_arm(A()) == 0
+
+
+def _run_bench(args, env_extra=None, timeout=180):
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                            "MASTER_PORT", "LOCAL_WORLD_SIZE")}
+    env.update(env_extra or {})
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "bench.py")
+    return subprocess.run([sys.executable, path, *args], capture_output=True, text=True, timeout=timeout, env=env)
+
+
+def test_gpus_flag_self_launches_two_gloo_ranks():
+    # --gpus 2 without a launcher: bench.py re-runs itself under torch.distributed.run with two
+    # ranks; the launch check joins them over gloo and rank 0 reports the world size
+    r = _run_bench(["--gpus", "2", "--launch-check"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert lines == [{"launch_check": True, "n_gpus": 2, "max_rank": 1.0}]
+
+
+def test_gpus_flag_disagreeing_with_world_size_fails():
+    r = _run_bench(["--gpus", "2", "--launch-check"], {"WORLD_SIZE": "1", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr

@@ -127,14 +127,69 @@ def test_gptq_weights_in_the_gemm(orc):
     assert e_gptq < e_rtn, (float(e_gptq), float(e_rtn))
 
 
-def test_hessian_factor_helper_matches_oracle(orc):
-    # the library's float64 preparation of U against the oracle's
-    K = 256
-    x = si.gptq_calibration(51, 2 * K, K)
-    for had in (0, 16, 32):
-        got = fl.gptq_hessian_factor(torch.from_numpy(x).to(DEV), had).cpu().numpy()
-        ref = orc.gptq_hessian_factor(x, had)
-        assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+def _definition_hinv(x, b, damp=0.01):
+    """H^-1 of the blockwise-rotated x in binary64, written out from the definition (scipy's
+    Sylvester Hadamard matrix, an explicit inverse)."""
+    import scipy.linalg
+    x = np.asarray(x, np.float64)
+    T, K = x.shape
+    if b:
+        x = x @ np.kron(np.eye(K // b), scipy.linalg.hadamard(b) / np.sqrt(b)).T
+    return np.linalg.inv(x.T @ x + damp * np.mean(np.sum(x * x, axis=0)) * np.eye(K))
+
+
+@pytest.mark.parametrize("K,T", [(64, 128), (256, 512), (320, 100), (1024, 2048 + 37)])
+@pytest.mark.parametrize("had", [0, 16, 32])
+def test_hessian_factor_matches_oracle(orc, K, T, had):
+    # the library's binary64 preparation of U against the oracle's, to 1e-5 max|U|; T < K (a
+    # rank-deficient Gram made definite by the damping) and a ragged T included; u is written
+    # into a poisoned buffer with a row stride wider than K
+    x = si.gptq_calibration(51 + K + had, T, K)
+    u = torch.full((K, K + 8), float("nan"), dtype=torch.float32, device=DEV)
+    got = fl.gptq_hessian_factor(torch.from_numpy(x).to(DEV), had, out=u[:, :K])
+    status_ok()
+    got = got.cpu().numpy()
+    assert np.all(np.isnan(u[:, K:].cpu().numpy()))  # nothing written past the row
+    ref = orc.gptq_hessian_factor(x, had)
+    assert np.all(np.tril(got, -1) == 0) and np.all(np.diag(got) > 0)
+    assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+    hinv = _definition_hinv(x, had)
+    g64 = got.astype(np.float64)
+    assert np.abs(g64.T @ g64 - hinv).max() <= 1e-5 * np.abs(hinv).max()
+
+
+@pytest.mark.slow
+def test_hessian_factor_prefill_size(orc):
+    # the size the bench prepares: K = 4096 with 8192 calibration tokens, H16
+    K = si.PREFILL["K"]
+    x = si.gptq_calibration(7, 2 * K, K)
+    got = fl.gptq_hessian_factor(torch.from_numpy(x).to(DEV), 16).cpu().numpy()
+    status_ok()
+    ref = orc.gptq_hessian_factor(x, 16)
+    assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+def test_hessian_factor_reports_a_singular_hessian():
+    # all-zero activations without damping: H = 0 has no Cholesky factor
+    x = torch.zeros(128, 64, dtype=torch.float64, device=DEV)
+    fl.gptq_hessian_factor(x, 16, damp=0.0)
+    assert fl.device_status() == 9  # FP4LIN_ERR_NUMERIC
+    assert fl.device_status() == 0
+
+
+def test_hessian_factor_feeds_gptq_like_the_oracle_factor(orc):
+    # the whole MR-GPTQ path through the library: the library's U is the oracle's to 1e-5 max|U|,
+    # and GPTQ with it gives the oracle's GPTQ codes for that same U, byte for byte
+    K, N = 128, 64
+    x = si.gptq_calibration(61, 2 * K, K)
+    w = si.normal_bf16(62, N, K, std=0.02)
+    u_lib = fl.gptq_hessian_factor(torch.from_numpy(x).to(DEV), 16)
+    u_orc = orc.gptq_hessian_factor(x, 16)
+    c, s, g = fl.gptq_quantize(w.to(DEV), u_lib, "nvfp4", 16)
+    status_ok()
+    oc, osf, og = orc.gptq(w, u_lib.cpu().numpy(), "nvfp4", 16)
+    assert_bytes_equal(c.cpu().numpy(), oc, "codes with the library's U")
+    assert np.abs(u_lib.cpu().numpy() - u_orc).max() <= 1e-5 * np.abs(u_orc).max()
 
 
 @pytest.mark.slow

@@ -62,6 +62,21 @@ def test_no_alloc_prefill_activations():
     assert torch.equal(c, rc) and torch.equal(s, rs) and torch.equal(g, rg)
 
 
+def test_python_wrapper_matches_c_abi_call():
+    # the binding's nvfp4_quantize_noalloc (argument checks, then the same C call) gives the
+    # bytes of the direct C-ABI call
+    x = si.student_t_bf16(73, 257, 2048).to(DEV)
+    c, s, g = _no_alloc(x, 16)
+    wc = torch.full_like(c, 0x55)
+    ws = torch.full_like(s, 0x11)
+    wg = torch.full((1,), -2.0, dtype=torch.float32, device=DEV)
+    fl.nvfp4_quantize_noalloc(x, 16, wg, wc, ws)
+    assert fl.device_status() == 0
+    assert torch.equal(wc, c) and torch.equal(ws, s) and torch.equal(wg, g)
+    with pytest.raises(ValueError):
+        fl.nvfp4_quantize_noalloc(x, 16, wg, wc[:-1], ws)  # a short codes buffer never reaches the C call
+
+
 def test_no_alloc_rejects_bad_arguments():
     L = fl.lib()
     P = 0x10000
