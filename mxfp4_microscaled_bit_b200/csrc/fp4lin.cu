@@ -312,9 +312,8 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
 }
 
 // Which kernel runs a GEMM of 256-column tiles that needs no K split: the one-CTA kernel
-// unless FP4LIN_GEMM_KERNEL=pair selects the CTA-pair kernel.  Both give identical results;
-// on the 8192 x 14336 x 4096 prefill product the one-CTA kernel is about 9% faster, since
-// both are limited by the scale copies into TMEM, which the pair does not reduce per SM.
+// unless FP4LIN_GEMM_KERNEL=pair selects the CTA-pair kernel.  Both give identical results
+// and, on the 8192 x 14336 x 4096 prefill product, times within a few per cent of each other.
 bool use_pair_kernel(const GemmPlan &pl)
 {
     if (pl.bn != 256 || pl.splits != 1)

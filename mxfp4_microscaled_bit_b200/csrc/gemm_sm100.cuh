@@ -11,9 +11,11 @@
 //   warp 0      TMA producer: code tiles by cp.async.bulk.tensor (128-byte
 //               swizzle), scale atoms by cp.async.bulk, into a STAGES-deep
 //               ring of shared-memory stages guarded by mbarriers.
-//   warp 1      owns TMEM; lane 0 copies each stage's scale atoms into TMEM
-//               (tcgen05.cp 32x128b.warpx4) and issues the block-scaled MMAs
-//               (128 x BN x 64 each) into a TMEM accumulator.
+//   warp 1      owns TMEM; the whole warp runs the issue loop (converged, polling
+//               the barriers) and one elected lane issues each instruction: the
+//               copies of a stage's scale atoms into TMEM (tcgen05.cp
+//               32x128b.warpx4) and the block-scaled MMAs (128 x BN x 64 each)
+//               into a TMEM accumulator.
 //   warps 2..9  epilogue: tcgen05.ld the accumulator into registers, release
 //               it at once, then scale by g_a*g_w, round to bf16 and store
 //               (or store fp32 partials when K is split across CTAs).
@@ -116,6 +118,33 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
+// Wait for the phase of `bar` with parity `parity` with every lane of the warp polling it (no
+// suspend hint): the form for warps that issue tcgen05 instructions as a converged warp and for
+// the epilogue's accumulator wait.  Every lane sees the same barrier state, the same clock and
+// the same flag, so the lanes stay together and agree on the outcome; lane 0 records a timeout.
+// Returns false when the wait gave up (after WAIT_LIMIT_NS, or once another role raised *abort).
+__device__ __forceinline__ bool warp_poll(uint64_t *bar, uint32_t parity, volatile int *abort, int lane)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 7u) == 0u) {
+            if (*abort)
+                return false;
+            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                if (lane == 0) {
+                    report_error(FP4LIN_ERR_TIMEOUT);
+                    *abort = 1;
+                }
+                return false;
+            }
+        }
+    }
+}
+
 // Diagnostic of the expiry path of wait_bounded, the wait every pipeline role
 // uses.  Two single-arrival barriers; lane 0 of warp w waits on barrier w.
 // Warp 1 waits with limit_ns, warp 0 with the kernel limit but honouring the
@@ -175,6 +204,47 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar)
 __device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t sdesc)
 {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// The same three instructions for a converged warp: every lane executes the call with the
+// same operands and one lane, chosen by elect.sync inside the asm, issues the instruction.
+// Issued this way the scale copies cost the tensor pipe almost nothing (a 128 x 256 x 64 MMA
+// with its three copies takes ~132 cycles, against ~225 when one lane of an otherwise idle
+// warp issues the same sequence: the operands then reach the issue unit through per-thread
+// registers).  Every lane of the warp must make the call.
+__device__ __forceinline__ void tc_cp_atom_w(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+                 "l"(sdesc)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_w(uint64_t *bar)
+{
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+template <bool NV>
+__device__ __forceinline__ void tc_mma_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                         uint32_t sfb, uint32_t acc)
+{
+    if constexpr (NV) {
+        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                         d),
+                     "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+                     : "memory");
+    } else {
+        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                         d),
+                     "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+                     : "memory");
+    }
 }
 
 template <bool NV>
@@ -553,8 +623,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer (one thread)
-        if (lane == 0) {
+        // ---------------------------------------------------------------- MMA issuer (one warp)
+        // The whole warp runs the loop on warp-uniform values and polls the barriers together
+        // (a suspending wait here costs far more than it saves), and one elected lane issues
+        // each tcgen05 instruction.
+        {
             const uint32_t tm_sf = tmem_base + C::NUM_ACC * C::BN;
             int stage = 0;
             uint32_t phase = 0, sfsel = 0;  // sfsel alternates the scale region every k-tile
@@ -566,14 +639,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
                 const int acc = it % C::NUM_ACC;
                 const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
-                if (!(ok = wait_bar(&acc_empty[acc], acc_phase ^ 1u, abort)))
+                if (!(ok = warp_poll(&acc_empty[acc], acc_phase ^ 1u, abort, lane)))
                     break;
                 tc_fence_after();  // order the epilogue's TMEM reads before these MMAs
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
                 // a 64-row B tile reads the second half of its 128-row scale atom at column +2
                 const uint32_t sfb_off = (C::BN == 64 && (((int64_t)nt * 64) & 127)) ? 2u : 0u;
                 for (int kt = kt0; kt < kt1; ++kt) {
-                    if (!(ok = wait_bar(&full[stage], phase, abort)))
+                    if (!(ok = warp_poll(&full[stage], phase, abort, lane)))
                         break;
                     const int mmas = stage_mmas<C>(p.K, kt);
                     uint8_t *sA = smem + stage * C::STAGE_BYTES;
@@ -584,20 +657,24 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     sfsel ^= 1u;
                     const uint32_t tm_sfb = tm_sfa + C::SFA_COLS;
                     const uint64_t dA = desc_sw128(smem_u32(sA)), dB = desc_sw128(smem_u32(sB));
-                    for (int kb = 0; kb < mmas; ++kb) {
+#pragma unroll
+                    for (int kb = 0; kb < C::BK / C::MMA_K; ++kb) {
+                        if (kb >= mmas)
+                            break;
                         // copy an atom's scales just before the first MMA that reads them, so the
                         // copies of k-block kb+1 overlap the MMA of k-block kb
                         const int a = C::NV ? kb : kb >> 1;
                         if (C::NV || (kb & 1) == 0) {
-                            tc_cp_atom(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
+                            tc_cp_atom_w(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
                             if constexpr (C::FUSEQ) {  // one copy per two k-blocks (see fuseq_store)
                                 if ((kb & 1) == 0)
-                                    tc_cp_atom(tm_sfb + (kb >> 1) * 4, desc_sf_atom(smem_u32(sSFB + (kb >> 1) * 512)));
+                                    tc_cp_atom_w(tm_sfb + (kb >> 1) * 4,
+                                                 desc_sf_atom(smem_u32(sSFB + (kb >> 1) * 512)));
                             } else {
 #pragma unroll
                                 for (int rt = 0; rt < C::RT; ++rt)
-                                    tc_cp_atom(tm_sfb + a * C::RT * 4 + rt * 4,
-                                               desc_sf_atom(smem_u32(sSFB + (rt * C::APK + a) * 512)));
+                                    tc_cp_atom_w(tm_sfb + a * C::RT * 4 + rt * 4,
+                                                 desc_sf_atom(smem_u32(sSFB + (rt * C::APK + a) * 512)));
                             }
                         }
                         uint32_t sfa, sfb, idesc;
@@ -615,10 +692,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             idesc = C::IDESC | (byte << 29) | (byte << 4);
                         }
                         // advance 64 FP4 values = 32 bytes inside the swizzled rows
-                        tc_mma<C::NV>(d_tmem, dA + (uint64_t)(kb * 2), dB + (uint64_t)(kb * 2), idesc, sfa, sfb,
-                                      (kt > kt0 || kb > 0) ? 1u : 0u);
+                        tc_mma_w<C::NV>(d_tmem, dA + (uint64_t)(kb * 2), dB + (uint64_t)(kb * 2), idesc, sfa, sfb,
+                                        (kt > kt0 || kb > 0) ? 1u : 0u);
                     }
-                    tc_commit(&empty[stage]);
+                    tc_commit_w(&empty[stage]);
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -626,11 +703,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(&acc_full[acc]);
+                tc_commit_w(&acc_full[acc]);
             }
             // every MMA this CTA issued has completed before TMEM is freed
-            tc_commit(done_bar);
-            wait_bounded(done_bar, 0, abort, false);
+            tc_commit_w(done_bar);
+            if (lane == 0)
+                wait_bounded(done_bar, 0, abort, false);
         }
         __syncwarp();
     } else {
@@ -770,10 +848,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
             const int acc = it % C::NUM_ACC;
             const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
-            // one warp waits on the accumulator; the others sleep in a named barrier (they issue
-            // nothing meanwhile, so the MMA-issuing warp keeps the SM's issue slots)
+            // one warp polls the accumulator barrier; the others sleep in a named barrier (they
+            // issue nothing meanwhile, so the MMA-issuing warp keeps the SM's issue slots)
             if (warp == 2) {
-                const bool okw = warp_wait(&acc_full[acc], acc_phase, abort, lane);
+                const bool okw = warp_poll(&acc_full[acc], acc_phase, abort, lane);
                 if (lane == 0)
                     epi_ok[it & 1] = okw ? 1 : 0;
             }

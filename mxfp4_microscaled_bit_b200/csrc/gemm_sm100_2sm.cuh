@@ -4,11 +4,10 @@
 // accumulator in its TMEM; the pair's tensor cores read both halves of B, so
 // per SM the operand traffic per FLOP drops by a third against the one-CTA
 // 128 x 256 tile, and a stage shrinks from 54 KB to 38 KB (five stages).
-// Operand feeding is not what limits the block-scaled GEMM on sm_100a, though:
-// each SM still writes the same scale bytes into TMEM per MMA (scale B for all
-// 256 columns, replicated in the four lane quadrants), and those writes stall
-// the MMA pipe.  So this kernel gives the same results as the one-CTA kernel,
-// a little slower, and runs only when FP4LIN_GEMM_KERNEL=pair asks for it.
+// Both kernels issue their tcgen05 instructions from a converged warp (see tc_mma_w);
+// measured on the 8192 x 14336 x 4096 prefill product the pair is within a few per cent
+// of the one-CTA kernel (faster for MXFP4, level for NVFP4), so it gives the same results
+// and runs only when FP4LIN_GEMM_KERNEL=pair asks for it.
 //
 // Roles (320 threads per CTA, both CTAs):
 //   warp 0 lane 0   producer: TMA loads of this CTA's A half, B half, scale A
@@ -107,6 +106,72 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t *bar)
 __device__ __forceinline__ void tc_cp_atom_pair(uint32_t taddr, uint64_t sdesc)
 {
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Converged-warp forms (every lane of the issuing warp makes the call, one elected lane issues;
+// see tc_mma_w in gemm_sm100.cuh).
+__device__ __forceinline__ void tc_commit_pair_w(uint64_t *bar)
+{
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "h"((uint16_t)3)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_cp_atom_pair_w(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr),
+                 "l"(sdesc)
+                 : "memory");
+}
+
+template <bool NV>
+__device__ __forceinline__ void tc_mma_pair_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                              uint32_t sfb, uint32_t acc)
+{
+    if constexpr (NV) {
+        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                         d),
+                     "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+                     : "memory");
+    } else {
+        asm volatile("{\n\t.reg .pred p, e;\n\tsetp.ne.b32 p, %4, 0;\n\telect.sync _|e, 0xffffffff;\n\t"
+                     "@e tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+                         d),
+                     "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+                     : "memory");
+    }
+}
+
+// warp_poll with cluster-scope acquire (the barrier's arrivals come from the peer CTA too).
+__device__ __forceinline__ bool warp_poll_cluster(uint64_t *bar, uint32_t parity, volatile int *abort, int lane)
+{
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(ok)
+                     : "r"(smem_u32(bar)), "r"(parity)
+                     : "memory");
+        if (ok)
+            return true;
+        if ((it & 7u) == 7u) {
+            if (*abort)
+                return false;
+            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                if (lane == 0) {
+                    report_error(FP4LIN_ERR_TIMEOUT);
+                    *abort = 1;
+                }
+                return false;
+            }
+        }
+    }
 }
 
 template <bool NV>
@@ -268,19 +333,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer (leader, one thread)
-        if (lane == 0 && rank == 0) {
+        // ---------------------------------------------------------------- MMA issuer (leader, one warp)
+        // The whole warp polls the barriers and runs the loop; one elected lane issues.
+        if (rank == 0) {
             const uint32_t tm_sf = tmem_base + C::BN;
             int stage = 0;
             uint32_t phase = 0, sfsel = 0;
             int it = 0;
             bool ok = true;
             for (int64_t w = pair; w < p.work && ok; w += npairs, ++it) {
-                if (!(ok = wait_bounded_cluster(acc_empty, ((uint32_t)it & 1u) ^ 1u, abort)))
+                if (!(ok = warp_poll_cluster(acc_empty, ((uint32_t)it & 1u) ^ 1u, abort, lane)))
                     break;
                 tc_fence_after();
                 for (int kt = 0; kt < p.nk; ++kt) {
-                    if (!(ok = wait_bar(&full[stage], phase, abort)))
+                    if (!(ok = warp_poll(&full[stage], phase, abort, lane)))
                         break;
                     const int mmas = stage_mmas<C>(p.K, kt);
                     uint8_t *sA = smem + stage * C::STAGE_BYTES;
@@ -291,13 +357,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                     sfsel ^= 1u;
                     const uint32_t tm_sfb = tm_sfa + C::SFA_COLS;
                     const uint64_t dA = desc_sw128(smem_u32(sA)), dB = desc_sw128(smem_u32(sB));
-                    for (int kb = 0; kb < mmas; ++kb) {
+#pragma unroll
+                    for (int kb = 0; kb < C::BK / C::MMA_K; ++kb) {
+                        if (kb >= mmas)
+                            break;
                         const int a = C::NV ? kb : kb >> 1;
                         if (C::NV || (kb & 1) == 0) {
                             // each CTA copies its own scale A atom and both 128-row scale B atoms
-                            tc_cp_atom_pair(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
-                            tc_cp_atom_pair(tm_sfb + a * 8, desc_sf_atom(smem_u32(sSFB + a * 512)));
-                            tc_cp_atom_pair(tm_sfb + a * 8 + 4, desc_sf_atom(smem_u32(sSFB + (C::APK + a) * 512)));
+                            tc_cp_atom_pair_w(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
+                            tc_cp_atom_pair_w(tm_sfb + a * 8, desc_sf_atom(smem_u32(sSFB + a * 512)));
+                            tc_cp_atom_pair_w(tm_sfb + a * 8 + 4, desc_sf_atom(smem_u32(sSFB + (C::APK + a) * 512)));
                         }
                         uint32_t sfa, sfb, idesc;
                         if (C::NV) {
@@ -310,10 +379,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                             sfb = (tm_sfb + a * 8) | (byte << 30);
                             idesc = C::IDESC | (byte << 29) | (byte << 4);
                         }
-                        tc_mma_pair<C::NV>(tmem_base, dA + (uint64_t)(kb * 2), dB + (uint64_t)(kb * 2), idesc, sfa,
-                                           sfb, (kt > 0 || kb > 0) ? 1u : 0u);
+                        tc_mma_pair_w<C::NV>(tmem_base, dA + (uint64_t)(kb * 2), dB + (uint64_t)(kb * 2), idesc, sfa,
+                                             sfb, (kt > 0 || kb > 0) ? 1u : 0u);
                     }
-                    tc_commit_pair(&empty[stage]);
+                    tc_commit_pair_w(&empty[stage]);
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -321,9 +390,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit_pair(acc_full);
+                tc_commit_pair_w(acc_full);
             }
-            tc_commit_pair(done_bar);
+            tc_commit_pair_w(done_bar);
         }
         // both CTAs: every MMA of the pair has completed before TMEM or shared memory is released
         if (lane == 0)
@@ -338,7 +407,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
         for (int64_t w = pair; w < p.work; w += npairs, ++it) {
             int mt, nt;
             pair_tile_coords(p, w, mt, nt);
-            if (!warp_wait(acc_full, (uint32_t)it & 1u, abort, lane))
+            if (!warp_poll(acc_full, (uint32_t)it & 1u, abort, lane))
                 break;
             tc_fence_after();
             float v[C::COLS_PER_WARP];
