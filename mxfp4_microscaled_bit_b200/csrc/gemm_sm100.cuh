@@ -333,7 +333,9 @@ struct GemmCfg {
     static constexpr int BK = 256;                        // elements per stage (128 code bytes per row)
     static constexpr int MMA_K = 64;
     static constexpr int APK = NV ? BK / 64 : BK / 128;   // scale atoms per 128 rows per stage
-    static constexpr int RT = BN <= 128 ? 1 : BN / 128;   // 128-row scale tiles per B stage
+    // 128-row scale tiles per B stage: a tile of BN rows starting at row BN * nt meets at most
+    // this many of the weight scale layout's 128-row tiles
+    static constexpr int RT = BN <= 128 ? 1 : (BN + 127) / 128;
     static constexpr int A_BYTES = BM * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int SFA_BYTES = APK * 512;
@@ -370,6 +372,7 @@ struct GemmParams {
     float *ws;                  // split-K partials [splits, M, ldw] (splits > 1)
     int64_t M, N, K, ldy, ldw;
     int64_t katoms;             // scale atoms per 128-row tile along K
+    int64_t sfb_rtiles;         // 128-row tiles of the B scale buffer (ceil(N / 128))
     int num_mt, num_nt, nk, kps, splits;
     int64_t work;               // num_mt * num_nt * splits
     // Optional NVFP4 quantisation of the bf16 output for the next layer (qc null: off):
@@ -591,10 +594,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     uint8_t *sB = sA + C::A_BYTES;
                     uint8_t *sSFA = sB + C::B_BYTES;
                     uint8_t *sSFB = sSFA + C::SFA_BYTES;
+                    // B scale row-tiles of this stage that exist (the last tile may reach past them)
+                    const int rts = (int)min((int64_t)C::RT, p.sfb_rtiles - brt0);
                     if constexpr (C::FUSEQ)  // the activation half of the stage comes from the epilogue warps
                         mbar_expect_tx(&full[stage], C::A_BYTES + atoms * 512);
                     else
-                        mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + C::RT));
+                        mbar_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES + atoms * 512 * (1 + rts));
                     armed |= 1u << stage;
                     armed_phase = (armed_phase & ~(1u << stage)) | (phase << stage);
                     if (p.a_tiled)
@@ -607,8 +612,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         tma_load_2d(sB, &tmB, &full[stage], kt * 128, nt * C::BN);
 #pragma unroll
                         for (int rt = 0; rt < C::RT; ++rt)
-                            bulk_load(sSFB + rt * C::APK * 512, p.sfb + ((brt0 + rt) * p.katoms + ka) * 512,
-                                      atoms * 512, &full[stage]);
+                            if (rt < rts)
+                                bulk_load(sSFB + rt * C::APK * 512, p.sfb + ((brt0 + rt) * p.katoms + ka) * 512,
+                                          atoms * 512, &full[stage]);
                     }
                     if (++stage == C::STAGES) {
                         stage = 0;
@@ -643,8 +649,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     break;
                 tc_fence_after();  // order the epilogue's TMEM reads before these MMAs
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
-                // a 64-row B tile reads the second half of its 128-row scale atom at column +2
-                const uint32_t sfb_off = (C::BN == 64 && (((int64_t)nt * 64) & 127)) ? 2u : 0u;
+                // a B tile starting 64 rows into a 128-row scale atom (BN = 64) reads its scales
+                // from the atom's column +2: 32 rows per TMEM column of the atom
+                const uint32_t sfb_off = (uint32_t)((((int64_t)nt * C::BN) & 127) >> 5);
                 for (int kt = kt0; kt < kt1; ++kt) {
                     if (!(ok = warp_poll(&full[stage], phase, abort, lane)))
                         break;
