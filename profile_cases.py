@@ -7,7 +7,7 @@ the 126 MB L2 but hold at most a few GB on the device.
 cases: gemm_prefill (8192 x 14336 x 4096 NVFP4, 16-wide rotation), gemm_mxfp4,
 gemm_decode (16 x 14336 x 4096), quant_prefill (8192 x 4096 rotated, dynamic
 scale; _static: the tensor scale given; _static_h0: given, no rotation),
-kv_load (8 x 8 x 32768 x 128 cache to FP8), kv_store, kv_attention (decode
+kv_load (8 x 8 x 32768 x 128 cache to FP8; --kv-batch sets the 8 sequences), kv_store, kv_attention (decode
 attention over the same 8 x 8 caches, G = 4), quant_mse (the 14336 x 4096 weight,
 MSE-optimal scales), gemm_quant (the prefill GEMM with its output NVFP4-encoded),
 linear_decode (16 x 14336 x 4096 with the activation quantiser inside the GEMM),
@@ -35,6 +35,8 @@ def main():
                              "quant_prefill_static_h0", "kv_load", "kv_store", "kv_attention", "quant_mse",
                              "gemm_quant", "linear_decode", "gptq"])
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--kv-batch", type=int, default=8,
+                    help="sequences in the kv_* cases' cache (8 x 8 x 32768 x 128 by default)")
     ap.add_argument("--time-cold", choices=["write", "read"], default=None,
                     help="time each call with CUDA events after flushing the L2 by writing (or reading) "
                          "512 MiB; print the mean")
@@ -95,7 +97,7 @@ def main():
         ca, sa, ga = fl.nvfp4_quantize(A)
         fn = lambda: fl.nvfp4_gemm(ca, sa, ga, w.codes, w.scales, w.g)  # noqa: E731
     else:
-        B, H, L, D = 8, 8, si.KVCACHE["L"], si.KVCACHE["D"]
+        B, H, L, D = a.kv_batch, 8, si.KVCACHE["L"], si.KVCACHE["D"]
         x = torch.empty(B, H, L, D, dtype=torch.bfloat16)
         for b in range(B):
             for h in range(H):
