@@ -936,10 +936,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int64_t n0 = (int64_t)nt * C::BN + half * C::COLS_PER_WARP;
             if (m < p.M) {
                 if (p.splits == 1) {
-                    // round once to bf16, in place: the stored y and the quantised y agree
 #pragma unroll
                     for (int c = 0; c < C::COLS_PER_WARP; ++c)
-                        v[c] = __bfloat162float(__float2bfloat16_rn(__fmul_rn(v[c], gg)));
+                        v[c] = __fmul_rn(v[c], gg);
+                    if (p.qc) {
+                        // round once to bf16, in place: the stored y and the quantised y agree
+#pragma unroll
+                        for (int c = 0; c < C::COLS_PER_WARP; ++c)
+                            v[c] = __bfloat162float(__float2bfloat16_rn(v[c]));
+                    }
                     if (p.y) {
                         __nv_bfloat16 *yr = p.y + m * p.ldy;
 #pragma unroll
