@@ -316,15 +316,22 @@ int launch_gemm_cfg(DeviceInfo *dev, int attr_slot, const GemmPlan &pl, const ui
     return FP4LIN_OK;
 }
 
-// Which kernel runs a GEMM of 256-column tiles that needs no K split: the one-CTA kernel
-// unless FP4LIN_GEMM_KERNEL=pair selects the CTA-pair kernel.  Both give identical results
-// and, on the 8192 x 14336 x 4096 prefill product, times within a few per cent of each other.
-bool use_pair_kernel(const GemmPlan &pl)
+// Which kernel runs a GEMM of 256-column tiles that needs no K split: the CTA-pair kernel
+// (256 x 256 tiles over two SMs) once M fills a pair's 256 rows, else the one-CTA kernel;
+// FP4LIN_GEMM_KERNEL=single or =pair forces one.  Both give identical results.  On the
+// 8192 x 14336 x 4096 prefill product the pair takes 212 us (NVFP4) and 189 us (MXFP4)
+// against the one-CTA kernel's 228 and 206 us: per SM it reads a third less operand data
+// from shared memory per FLOP.
+bool use_pair_kernel(const GemmPlan &pl, int64_t M)
 {
     if (pl.bn != 256 || pl.splits != 1)
         return false;
     const char *e = getenv("FP4LIN_GEMM_KERNEL");
-    return e && strcmp(e, "pair") == 0;
+    if (e && strcmp(e, "single") == 0)
+        return false;
+    if (e && strcmp(e, "pair") == 0)
+        return true;
+    return M >= 256;
 }
 
 template <class C>
@@ -535,7 +542,7 @@ int gemm_entry(bool nv, const uint8_t *a_codes, const uint8_t *a_scales, const f
         return launch_gemm_cfg<GemmCfg<16, false, true>>(dev, 5, pl, w_codes, w_scales, nullptr, a_codes, a_scales,
                                                          nullptr, y, N, M, K, ldy, ws, s, qo);
     }
-    if (!quant && use_pair_kernel(pl)) {
+    if (!quant && use_pair_kernel(pl, M)) {
         if (nv)
             return launch_gemm_pair<Gemm2Cfg<true>>(dev, 0, a_codes, a_scales, g_a, w_codes, w_scales, g_w, y, M, N,
                                                     K, ldy, s);

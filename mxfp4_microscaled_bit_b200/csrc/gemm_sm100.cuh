@@ -11,14 +11,18 @@
 //   warp 0      TMA producer: code tiles by cp.async.bulk.tensor (128-byte
 //               swizzle), scale atoms by cp.async.bulk, into a STAGES-deep
 //               ring of shared-memory stages guarded by mbarriers.
-//   warp 1      owns TMEM; the whole warp runs the issue loop (converged, polling
-//               the barriers) and one elected lane issues each instruction: the
-//               copies of a stage's scale atoms into TMEM (tcgen05.cp
-//               32x128b.warpx4) and the block-scaled MMAs (128 x BN x 64 each)
-//               into a TMEM accumulator.
+//   warp 1      owns TMEM; the whole warp runs the issue loop (converged) and one
+//               elected lane issues each instruction: the copies of a stage's
+//               scale atoms into TMEM (tcgen05.cp 32x128b.warpx4) and the
+//               block-scaled MMAs (128 x BN x 64 each) into a TMEM accumulator.
+//               It waits on no mbarrier itself: between tensor-core instructions
+//               such a wait stalls the issue far longer than a named barrier.
 //   warps 2..9  epilogue: tcgen05.ld the accumulator into registers, release
 //               it at once, then scale by g_a*g_w, round to bf16 and store
-//               (or store fp32 partials when K is split across CTAs).
+//               (256-bit stores; fp32 partials when K is split across CTAs).
+//   warp 10     waiter: polls the accumulator and stage barriers in the MMA
+//               warp's order, one step ahead of it, and meets it at a named
+//               barrier after each, passing on a wait that gave up.
 // Every mbarrier wait is bounded (WAIT_LIMIT_NS); on expiry the kernel
 // records FP4LIN_ERR_TIMEOUT, raises a CTA abort flag, waits (bounded) for
 // its own copies and MMAs, frees TMEM and returns.
@@ -143,6 +147,20 @@ __device__ __forceinline__ bool warp_poll(uint64_t *bar, uint32_t parity, volati
             }
         }
     }
+}
+
+// The MMA warp and its waiter warp meet at named barrier 2 (64 threads); the result is true
+// when either side passed true (a wait that gave up).  A named barrier costs the issuing warp
+// far less than an mbarrier wait of its own between its tensor-core instructions.
+__device__ __forceinline__ bool meet_or(bool fail)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\tbar.red.or.pred p, 2, 64, q;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(r)
+                 : "r"((uint32_t)fail)
+                 : "memory");
+    return r != 0;
 }
 
 // Diagnostic of the expiry path of wait_bounded, the wait every pipeline role
@@ -349,7 +367,8 @@ struct GemmCfg {
     static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128
                                    : TMEM_USED <= 256 ? 256 : 512;
     static constexpr int EPI_WARPS = 8;
-    static constexpr int THREADS = 64 + EPI_WARPS * 32;
+    static constexpr int WAITER_WARP = 2 + EPI_WARPS;    // waits on the MMA warp's barriers
+    static constexpr int THREADS = 64 + EPI_WARPS * 32 + 32;
     static constexpr int COLS_PER_WARP = BN / 2;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
@@ -630,9 +649,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer (one warp)
-        // The whole warp runs the loop on warp-uniform values and polls the barriers together
-        // (a suspending wait here costs far more than it saves), and one elected lane issues
-        // each tcgen05 instruction.
+        // The whole warp runs the loop on warp-uniform values and one elected lane issues each
+        // tcgen05 instruction.  The waiter warp does the barrier waits; this warp meets it at
+        // named barrier 2 before each tile and each k-tile.
         {
             const uint32_t tm_sf = tmem_base + C::NUM_ACC * C::BN;
             int stage = 0;
@@ -645,7 +664,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
                 const int acc = it % C::NUM_ACC;
                 const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
-                if (!(ok = warp_poll(&acc_empty[acc], acc_phase ^ 1u, abort, lane)))
+                if (!(ok = !meet_or(false)))  // the waiter saw the accumulator free
                     break;
                 tc_fence_after();  // order the epilogue's TMEM reads before these MMAs
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
@@ -653,7 +672,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 // from the atom's column +2: 32 rows per TMEM column of the atom
                 const uint32_t sfb_off = (uint32_t)((((int64_t)nt * C::BN) & 127) >> 5);
                 for (int kt = kt0; kt < kt1; ++kt) {
-                    if (!(ok = warp_poll(&full[stage], phase, abort, lane)))
+                    if (!(ok = !meet_or(false)))  // the waiter saw the stage full
                         break;
                     const int mmas = stage_mmas<C>(p.K, kt);
                     uint8_t *sA = smem + stage * C::STAGE_BYTES;
@@ -718,6 +737,36 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 wait_bounded(done_bar, 0, abort, false);
         }
         __syncwarp();
+    } else if (warp == C::WAITER_WARP) {
+        // ---------------------------------------------------------------- waiter (one warp)
+        // Walks the MMA warp's sequence of barrier waits -- per tile the accumulator, per k-tile
+        // the stage -- one step ahead of it, and meets it after each (named barrier 2, which also
+        // carries a failed wait to it).  Both leave at the same meeting.
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        bool ok = true;
+        for (int64_t w = blockIdx.x; w < p.work && ok; w += gridDim.x, ++it) {
+            int mt, nt, sp;
+            tile_coords(p, w, mt, nt, sp);
+            const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+            const int acc = it % C::NUM_ACC;
+            const uint32_t acc_phase = (uint32_t)(it / C::NUM_ACC) & 1u;
+            if (meet_or(!warp_poll(&acc_empty[acc], acc_phase ^ 1u, abort, lane))) {
+                ok = false;
+                break;
+            }
+            for (int kt = kt0; kt < kt1; ++kt) {
+                if (meet_or(!warp_poll(&full[stage], phase, abort, lane))) {
+                    ok = false;
+                    break;
+                }
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
     } else {
         // ---------------------------------------------------------------- epilogue
         const int quad = warp & 3;                       // TMEM lanes this warp may access
@@ -947,21 +996,37 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                     if (p.y) {
                         __nv_bfloat16 *yr = p.y + m * p.ldy;
+                        // 16 columns per 256-bit store where the row segment is 32-byte aligned
+                        const bool w32 = (reinterpret_cast<uintptr_t>(yr + n0) & 31) == 0;
 #pragma unroll
-                        for (int c = 0; c < C::COLS_PER_WARP; c += 8) {
+                        for (int c = 0; c < C::COLS_PER_WARP; c += 16) {
                             const int64_t n = n0 + c;
-                            if (n + 8 <= p.N) {
-                                uint32_t w4[4];
+                            if (w32 && n + 16 <= p.N) {
+                                uint32_t w8[8];
 #pragma unroll
-                                for (int j = 0; j < 4; ++j) {
+                                for (int j = 0; j < 8; ++j) {
                                     __nv_bfloat162 b2 = __floats2bfloat162_rn(v[c + 2 * j], v[c + 2 * j + 1]);
-                                    w4[j] = *reinterpret_cast<uint32_t *>(&b2);
+                                    w8[j] = *reinterpret_cast<uint32_t *>(&b2);
                                 }
-                                st_v4(yr + n, make_uint4(w4[0], w4[1], w4[2], w4[3]));
-                            } else {
-                                for (int j = 0; j < 8; ++j)
-                                    if (n + j < p.N)
-                                        yr[n + j] = __float2bfloat16_rn(v[c + j]);
+                                st_v8(yr + n, w8);
+                                continue;
+                            }
+#pragma unroll
+                            for (int h = 0; h < 16; h += 8) {
+                                if (n + h + 8 <= p.N) {
+                                    uint32_t w4[4];
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        __nv_bfloat162 b2 =
+                                            __floats2bfloat162_rn(v[c + h + 2 * j], v[c + h + 2 * j + 1]);
+                                        w4[j] = *reinterpret_cast<uint32_t *>(&b2);
+                                    }
+                                    st_v4(yr + n + h, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+                                } else {
+                                    for (int j = 0; j < 8; ++j)
+                                        if (n + h + j < p.N)
+                                            yr[n + h + j] = __float2bfloat16_rn(v[c + h + j]);
+                                }
                             }
                         }
                     }

@@ -4,21 +4,25 @@
 // accumulator in its TMEM; the pair's tensor cores read both halves of B, so
 // per SM the operand traffic per FLOP drops by a third against the one-CTA
 // 128 x 256 tile, and a stage shrinks from 54 KB to 38 KB (five stages).
-// Both kernels issue their tcgen05 instructions from a converged warp (see tc_mma_w);
-// measured on the 8192 x 14336 x 4096 prefill product the pair is within a few per cent
-// of the one-CTA kernel (faster for MXFP4, level for NVFP4), so it gives the same results
-// and runs only when FP4LIN_GEMM_KERNEL=pair asks for it.
+// Both kernels issue their tcgen05 instructions from a converged warp (see tc_mma_w) and
+// give the same results bit for bit.  On the 8192 x 14336 x 4096 prefill product the pair
+// takes 212 us (NVFP4) and 189 us (MXFP4), the one-CTA kernel 228 and 206 us, so the pair
+// runs every GEMM of 256-column tiles without a K split once M >= 256
+// (FP4LIN_GEMM_KERNEL=single or =pair forces either).
 //
-// Roles (320 threads per CTA, both CTAs):
+// Roles (352 threads per CTA, both CTAs):
 //   warp 0 lane 0   producer: TMA loads of this CTA's A half, B half, scale A
 //                   (its 128 rows) and scale B (all 256 N rows -- every CTA's
 //                   TMEM needs them), all completing on the LEADER's `full`
 //                   barrier (cta_group::2 form, peer bit of the address cleared);
 //   warp 1          TMEM (cta_group::2 alloc/dealloc in both CTAs); in the
-//                   leader, lane 0 issues the scale copies and MMAs for the pair
-//                   and commits, multicast to both CTAs' barriers;
+//                   leader, the converged warp issues (one elected lane) the scale
+//                   copies and MMAs for the pair and commits, multicast to both
+//                   CTAs' barriers;
 //   warps 2..9      epilogue of this CTA's 128 accumulator rows; they release
-//                   the accumulator by arriving on the leader's `acc_empty`.
+//                   the accumulator by arriving on the leader's `acc_empty`;
+//   warp 10         in the leader, waits on the barriers for the MMA warp and
+//                   meets it at a named barrier (as in the one-CTA kernel).
 // All waits are bounded as in the one-CTA kernel.  No load uses multicast.
 #pragma once
 
@@ -210,7 +214,8 @@ struct Gemm2Cfg {
     static constexpr int TMEM_USED = BN + 2 * SF_COLS;
     static constexpr int TMEM_COLS = 512;
     static constexpr int EPI_WARPS = 8;
-    static constexpr int THREADS = 64 + EPI_WARPS * 32;
+    static constexpr int WAITER_WARP = 2 + EPI_WARPS;    // the leader's barrier waits for its MMA warp
+    static constexpr int THREADS = 64 + EPI_WARPS * 32 + 32;
     static constexpr int COLS_PER_WARP = BN / 2;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
@@ -342,11 +347,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             int it = 0;
             bool ok = true;
             for (int64_t w = pair; w < p.work && ok; w += npairs, ++it) {
-                if (!(ok = warp_poll_cluster(acc_empty, ((uint32_t)it & 1u) ^ 1u, abort, lane)))
+                if (!(ok = !meet_or(false)))  // the waiter saw both CTAs' epilogues release the accumulator
                     break;
                 tc_fence_after();
                 for (int kt = 0; kt < p.nk; ++kt) {
-                    if (!(ok = warp_poll(&full[stage], phase, abort, lane)))
+                    if (!(ok = !meet_or(false)))  // the waiter saw both CTAs' stage bytes land
                         break;
                     const int mmas = stage_mmas<C>(p.K, kt);
                     uint8_t *sA = smem + stage * C::STAGE_BYTES;
@@ -398,6 +403,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
         if (lane == 0)
             wait_bounded(done_bar, 0, abort, false);
         __syncwarp();
+    } else if (warp == C::WAITER_WARP) {
+        // ---------------------------------------------------------------- waiter (leader, one warp)
+        // The MMA warp's barrier waits, one step ahead of it, each followed by a meeting at
+        // named barrier 2 that passes on a wait that gave up.
+        if (rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (int64_t w = pair; w < p.work && ok; w += npairs, ++it) {
+                if (meet_or(!warp_poll_cluster(acc_empty, ((uint32_t)it & 1u) ^ 1u, abort, lane))) {
+                    ok = false;
+                    break;
+                }
+                for (int kt = 0; kt < p.nk; ++kt) {
+                    if (meet_or(!warp_poll(&full[stage], phase, abort, lane))) {
+                        ok = false;
+                        break;
+                    }
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
     } else {
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const int quad = warp & 3;
@@ -424,22 +455,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             const int64_t n0 = (int64_t)nt * C::BN + half * C::COLS_PER_WARP;
             if (m < p.M) {
                 __nv_bfloat16 *yr = p.y + m * p.ldy;
+                // 16 columns per 256-bit store where the row segment is 32-byte aligned
+                const bool w32 = (reinterpret_cast<uintptr_t>(yr + n0) & 31) == 0;
 #pragma unroll
-                for (int c = 0; c < C::COLS_PER_WARP; c += 8) {
+                for (int c = 0; c < C::COLS_PER_WARP; c += 16) {
                     const int64_t n = n0 + c;
-                    if (n + 8 <= p.N) {
-                        uint32_t w4[4];
+                    if (w32 && n + 16 <= p.N) {
+                        uint32_t w8[8];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
+                        for (int j = 0; j < 8; ++j) {
                             __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(v[c + 2 * j], gg),
                                                                       __fmul_rn(v[c + 2 * j + 1], gg));
-                            w4[j] = *reinterpret_cast<uint32_t *>(&b2);
+                            w8[j] = *reinterpret_cast<uint32_t *>(&b2);
                         }
-                        st_v4(yr + n, make_uint4(w4[0], w4[1], w4[2], w4[3]));
-                    } else {
-                        for (int j = 0; j < 8; ++j)
-                            if (n + j < p.N)
-                                yr[n + j] = __float2bfloat16_rn(__fmul_rn(v[c + j], gg));
+                        st_v8(yr + n, w8);
+                        continue;
+                    }
+#pragma unroll
+                    for (int h = 0; h < 16; h += 8) {
+                        if (n + h + 8 <= p.N) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(v[c + h + 2 * j], gg),
+                                                                          __fmul_rn(v[c + h + 2 * j + 1], gg));
+                                w4[j] = *reinterpret_cast<uint32_t *>(&b2);
+                            }
+                            st_v4(yr + n + h, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+                        } else {
+                            for (int j = 0; j < 8; ++j)
+                                if (n + h + j < p.N)
+                                    yr[n + h + j] = __float2bfloat16_rn(__fmul_rn(v[c + h + j], gg));
+                        }
                     }
                 }
             }
