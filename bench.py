@@ -47,8 +47,8 @@ FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP
 # DRAM bytes (read + write) per step for a kernel, from one ncu capture of the current build
 # (summarised under profiles/); None where no capture covers the kernel as it stands.
 NCU_TRAFFIC = {
-    "gemm": 291.8e6,          # the 8192x14336x4096 prefill GEMM, one launch
-    "mxfp4_gemm": 275.2e6,    # the same product in MXFP4, one launch
+    "gemm": 308.7e6,          # the 8192x14336x4096 prefill GEMM (CTA-pair kernel), one launch
+    "mxfp4_gemm": None,       # the same product in MXFP4, one launch
     "kv_load_fp8": 6.511e9,   # 1627.6 MB per 32x8x32768x128 cache, x 2 (64 sequences) x 2 (K, V)
     "quantize": None,         # the capture covers the quantise pass only, not the amax pass
     "kv_store": None,
@@ -58,7 +58,6 @@ NCU_TRAFFIC_NOTE = {
     "kv_load_fp8": "DRAM bytes of a 32x8x32768x128 capture (reads 604.0 MB = the codes and scales once) scaled "
                    "x4 by the units processed; ~50 MB of that launch's writes were still in L2 when it ended "
                    "(written back after it), so the figure reads 3% below the 6.711 GB algorithmic bytes",
-    "mxfp4_gemm": "~9 MB of y still in L2 when the captured launch ended",
 }
 METRIC = "NVFP4 GEMM TFLOP/s (% dense FP4 peak); quantize/KV GB/s (% of HBM)"
 

@@ -7,18 +7,22 @@
 // M = 256: the leader issues one scale-A copy (each CTA copies its own 128 rows), one scale-B
 // copy and one MMA for 256 weight rows -- half the instructions per weight row.
 //
-// Measured, it is slower than the one-CTA form (16x14336x4096: 16.5 against 15.0 us): the
-// pair's instructions and its completions on the leader's barriers cost more each, so it runs
-// only when FP4LIN_DECODE_KERNEL=pair asks for it.  Its results are the same, bit for bit.
+// Measured, it is slower than the one-CTA form (16x14336x4096: 18.5 against 15.8 us, both
+// issuing from a converged warp with a waiter warp): the pair's completions on the leader's
+// barriers and its cluster-wide hand-offs cost more than the instructions it saves, so it
+// runs only when FP4LIN_DECODE_KERNEL=pair asks for it.  Its results are the same, bit for bit.
 //
-// Roles (320 threads per CTA, both CTAs of the pair):
+// Roles (352 threads per CTA, both CTAs of the pair):
 //   warp 0 lane 0   producer: TMA loads of this CTA's 128 weight rows, its 8 of the 16
 //                   activation rows, its weight scale atoms and all activation scale atoms
 //                   (every CTA's TMEM needs them), completing on the LEADER's `full` barrier;
-//   warp 1          TMEM (cta_group::2 alloc/dealloc); in the leader lane 0 issues the pair's
-//                   copies and MMAs and commits, multicast to both CTAs' barriers;
+//   warp 1          TMEM (cta_group::2 alloc/dealloc); in the leader the converged warp issues
+//                   (one elected lane) the pair's copies and MMAs and commits, multicast to
+//                   both CTAs' barriers;
 //   warps 2..9      epilogue of this CTA's 128 weight rows: y (transposed) or, with a K split,
-//                   binary32 partial sums for splitk_reduce_kernel.
+//                   binary32 partial sums for splitk_reduce_kernel;
+//   warp 10         in the leader, waits on the barriers for the MMA warp and meets it at a
+//                   named barrier.
 // Two accumulators (16 columns each) let a pair start its next item while the previous one
 // drains.  All waits are bounded.  No load uses multicast.
 #pragma once
@@ -46,7 +50,8 @@ struct GemmDecodePairCfg {
     static constexpr int TMEM_USED = NUM_ACC * BN + 2 * SF_COLS;
     static constexpr int TMEM_COLS = TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : 256;
     static constexpr int EPI_WARPS = 8;
-    static constexpr int THREADS = 64 + EPI_WARPS * 32;
+    static constexpr int WAITER_WARP = 2 + EPI_WARPS;    // the leader's barrier waits for its MMA warp
+    static constexpr int THREADS = 64 + EPI_WARPS * 32 + 32;
     static constexpr int COLS_PER_WARP = BN / 2;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
@@ -156,8 +161,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer (leader, one thread)
-        if (lane == 0 && rank == 0) {
+        // ---------------------------------------------------------------- MMA issuer (leader, one warp)
+        // The converged warp runs the loop and one elected lane issues; the waiter warp does the
+        // barrier waits and meets this warp at named barrier 2 (as in the prefill kernels).
+        if (rank == 0) {
             const uint32_t tm_sf = tmem_base + C::NUM_ACC * C::BN;
             int stage = 0;
             uint32_t phase = 0, sfsel = 0;
@@ -167,12 +174,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                 const int sp = (int)(w / p.num_mt);
                 const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
                 const int acc = it & 1;
-                if (!(ok = wait_bounded_cluster(&acc_empty[acc], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort)))
+                if (!(ok = !meet_or(false)))  // the waiter saw both CTAs' epilogues release the accumulator
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * C::BN;
                 for (int kt = kt0; kt < kt1; ++kt) {
-                    if (!(ok = wait_bar(&full[stage], phase, abort)))
+                    if (!(ok = !meet_or(false)))  // the waiter saw both CTAs' stage bytes land
                         break;
                     const int mmas = stage_mmas<C>(p.K, kt);
                     uint8_t *sA = smem + stage * C::STAGE_BYTES;
@@ -183,12 +190,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                     sfsel ^= 1u;
                     const uint32_t tm_sfb = tm_sfa + C::SFA_COLS;
                     const uint64_t dA = desc_sw128(smem_u32(sA)), dB = desc_sw128(smem_u32(sB));
-                    for (int kb = 0; kb < mmas; ++kb) {
+#pragma unroll
+                    for (int kb = 0; kb < C::BK / C::MMA_K; ++kb) {
+                        if (kb >= mmas)
+                            break;
                         const int a = C::NV ? kb : kb >> 1;
                         if (C::NV || (kb & 1) == 0) {
                             // each CTA copies its own weight scale atom and the activation scale atom
-                            tc_cp_atom_pair(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
-                            tc_cp_atom_pair(tm_sfb + a * 4, desc_sf_atom(smem_u32(sSFB + a * 512)));
+                            tc_cp_atom_pair_w(tm_sfa + a * 4, desc_sf_atom(smem_u32(sSFA + a * 512)));
+                            tc_cp_atom_pair_w(tm_sfb + a * 4, desc_sf_atom(smem_u32(sSFB + a * 512)));
                         }
                         uint32_t sfa, sfb, idesc;
                         if (C::NV) {
@@ -201,10 +211,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                             sfb = (tm_sfb + a * 4) | (byte << 30);
                             idesc = C::IDESC | (byte << 29) | (byte << 4);
                         }
-                        tc_mma_pair<C::NV>(d_tmem, dA + (uint64_t)(kb * 2), dB + (uint64_t)(kb * 2), idesc, sfa, sfb,
-                                           (kt > kt0 || kb > 0) ? 1u : 0u);
+                        tc_mma_pair_w<C::NV>(d_tmem, dA + (uint64_t)(kb * 2), dB + (uint64_t)(kb * 2), idesc, sfa,
+                                             sfb, (kt > kt0 || kb > 0) ? 1u : 0u);
                     }
-                    tc_commit_pair(&empty[stage]);
+                    tc_commit_pair_w(&empty[stage]);
                     if (++stage == C::STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -212,14 +222,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit_pair(&acc_full[acc]);
+                tc_commit_pair_w(&acc_full[acc]);
             }
-            tc_commit_pair(done_bar);
+            tc_commit_pair_w(done_bar);
         }
         // both CTAs: every MMA of the pair has completed before TMEM or shared memory is released
         if (lane == 0)
             wait_bounded(done_bar, 0, abort, false);
         __syncwarp();
+    } else if (warp == C::WAITER_WARP) {
+        // ---------------------------------------------------------------- waiter (leader, one warp)
+        if (rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (int64_t w = pair; w < p.work && ok; w += npairs, ++it) {
+                const int sp = (int)(w / p.num_mt);
+                const int kt0 = sp * p.kps, kt1 = min(p.nk, kt0 + p.kps);
+                const int acc = it & 1;
+                if (meet_or(!warp_poll_cluster(&acc_empty[acc], ((uint32_t)(it >> 1) & 1u) ^ 1u, abort, lane))) {
+                    ok = false;
+                    break;
+                }
+                for (int kt = kt0; kt < kt1; ++kt) {
+                    if (meet_or(!warp_poll(&full[stage], phase, abort, lane))) {
+                        ok = false;
+                        break;
+                    }
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+        }
     } else {
         // ---------------------------------------------------------------- epilogue (both CTAs)
         const int quad = warp & 3;
