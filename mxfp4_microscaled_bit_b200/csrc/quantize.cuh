@@ -67,7 +67,7 @@ __device__ __forceinline__ void fwht(float *v)
 // scalar; every stride h >= 2 pairs element 2m with 2m+h and 2m+1 with 2m+1+h, so the
 // pairs (v[2m], v[2m+1]) move together through add/sub.f32x2 -- the same IEEE operations
 // in the same order, two per instruction.  The 1/sqrt(B) scaling `s` is packed too.
-template <int B>
+template <int B, bool SCALE = true>
 __device__ __forceinline__ void fwht_scaled_packed(float *v, float s)
 {
 #pragma unroll
@@ -89,10 +89,16 @@ __device__ __forceinline__ void fwht_scaled_packed(float *v, float s)
                 P[m] = f2_add(a, b);
                 P[m + h2] = f2_sub(a, b);
             }
-    const uint64_t ss = f2_pack(s, s);
+    if constexpr (SCALE) {
+        const uint64_t ss = f2_pack(s, s);
 #pragma unroll
-    for (int m = 0; m < B / 2; ++m)
-        f2_unpack(f2_mul(P[m], ss), v[2 * m], v[2 * m + 1]);
+        for (int m = 0; m < B / 2; ++m)
+            f2_unpack(f2_mul(P[m], ss), v[2 * m], v[2 * m + 1]);
+    } else {
+#pragma unroll
+        for (int m = 0; m < B / 2; ++m)
+            f2_unpack(P[m], v[2 * m], v[2 * m + 1]);
+    }
 }
 
 // v[j] = RN(v[j] * s) for B values, two per packed instruction.
@@ -105,24 +111,47 @@ __device__ __forceinline__ void scale_packed(float *v, float s)
         f2_unpack(f2_mul(f2_pack(v[2 * m], v[2 * m + 1]), ss), v[2 * m], v[2 * m + 1]);
 }
 
+// max(a, b, c) in one instruction (the three-input form of max.f32; like fmaxf, a NaN input
+// is ignored).
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// max |v[i]| over B values: for B a multiple of 16 by three-input maxima (8 per 16 values).
 template <int B>
 __device__ __forceinline__ float abs_max(const float *v)
 {
     float m = 0.0f;
+    if constexpr (B % 16 != 0) {
 #pragma unroll
-    for (int i = 0; i < B; ++i)
-        m = fmaxf(m, fabsf(v[i]));
+        for (int i = 0; i < B; ++i)
+            m = fmaxf(m, fabsf(v[i]));
+        return m;
+    }
+#pragma unroll
+    for (int i = 0; i < B; i += 16) {
+        const float a = max3f(fabsf(v[i + 0]), fabsf(v[i + 1]), fabsf(v[i + 2]));
+        const float b = max3f(fabsf(v[i + 3]), fabsf(v[i + 4]), fabsf(v[i + 5]));
+        const float c = max3f(fabsf(v[i + 6]), fabsf(v[i + 7]), fabsf(v[i + 8]));
+        const float d = max3f(fabsf(v[i + 9]), fabsf(v[i + 10]), fabsf(v[i + 11]));
+        const float e = max3f(fabsf(v[i + 12]), fabsf(v[i + 13]), fabsf(v[i + 14]));
+        m = max3f(m, max3f(a, b, c), max3f(d, e, fabsf(v[i + 15])));
+    }
     return m;
 }
 
-// The (rotated, when HAD) values of one NVFP4 block: 16 bf16 in `raw`.
-template <bool HAD>
+// The (rotated, when HAD) values of one NVFP4 block: 16 bf16 in `raw`.  SCALE false leaves
+// out the rotation's final exact factor 1/4 (for a maximum, which can take it afterwards).
+template <bool HAD, bool SCALE = true>
 __device__ __forceinline__ void nvfp4_block_values(const uint32_t *raw, float *v)
 {
     bf16x8_to_f32(make_uint4(raw[0], raw[1], raw[2], raw[3]), v);
     bf16x8_to_f32(make_uint4(raw[4], raw[5], raw[6], raw[7]), v + 8);
     if (HAD)
-        fwht_scaled_packed<16>(v, 0.25f);  // 1/sqrt(16), exact
+        fwht_scaled_packed<16, SCALE>(v, 0.25f);  // 1/sqrt(16), exact
 }
 
 // The (rotated, when HAD) values of one MXFP4 block: 32 bf16 in `raw`.
@@ -190,11 +219,15 @@ __global__ void __launch_bounds__(QTHREADS) nvfp4_amax_kernel(QuantShape q, floa
 #pragma unroll
             for (int u = 0; u < QUNROLL; ++u) {
                 float v[16];
-                nvfp4_block_values<HAD>(raw[u], v);
+                nvfp4_block_values<HAD, false>(raw[u], v);
                 m = fmaxf(m, abs_max<16>(v));
             }
         }
     }
+    // the rotation's factor 1/4 on the maximum instead of on every value: x -> RN(x / 4) is
+    // non-decreasing and odd, so the maximum of the scaled magnitudes is the scaled maximum
+    if (HAD)
+        m = __fmul_rn(m, 0.25f);
 #pragma unroll
     for (int o = 16; o; o >>= 1)
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
