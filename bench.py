@@ -48,7 +48,7 @@ FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput (9 : 2.25 PFLOP
 # (summarised under profiles/); None where no capture covers the kernel as it stands.
 NCU_TRAFFIC = {
     "gemm": 308.7e6,          # the 8192x14336x4096 prefill GEMM (CTA-pair kernel), one launch
-    "mxfp4_gemm": None,       # the same product in MXFP4, one launch
+    "mxfp4_gemm": 293.7e6,    # the same product in MXFP4 (CTA-pair kernel), one launch
     "kv_load_fp8": 6.511e9,   # 1627.6 MB per 32x8x32768x128 cache, x 2 (64 sequences) x 2 (K, V)
     "quantize": None,         # the capture covers the quantise pass only, not the amax pass
     "kv_store": None,
