@@ -520,7 +520,7 @@ __device__ __forceinline__ void fuseq_load(const GemmParams &p, int kt, int et, 
 }
 
 __device__ __forceinline__ void fuseq_store(const GemmParams &p, uint8_t *sB, uint8_t *sSFB, int kt, int et,
-                                            const FuseRaw &x, float xg)
+                                            const FuseRaw &x, float xg, float c6, const float *s_rcp)
 {
     const int r = et >> 4, c = et & 15;
     uint32_t lo = 0u, hi = 0u, sf = 0u;
@@ -531,9 +531,10 @@ __device__ __forceinline__ void fuseq_store(const GemmParams &p, uint8_t *sB, ui
             nvfp4_block_values<true>(raw, v);
         else
             nvfp4_block_values<false>(raw, v);
-        float rcp;
-        sf = nvfp4_block_scale(abs_max<16>(v), xg, rcp);
-        scale_packed<16>(v, rcp);
+        // nvfp4_block_scale's byte and multiplier without a division: c6 and the table of
+        // 1/(dec(sf) xg) over the 256 scale bytes are computed once per CTA
+        sf = nvfp4_scale_code_fast(abs_max<16>(v), xg, c6);
+        scale_packed<16>(v, s_rcp[sf]);
         lo = pack_e2m1x8(v);
         hi = pack_e2m1x8(v + 8);
     }
@@ -776,6 +777,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         float xg = 0.0f;                                 // FUSEQ: the activations' tensor scale
         __shared__ float s_xred[C::EPI_WARPS];
         __shared__ float s_xg;
+        __shared__ float s_rcp[C::FUSEQ ? 256 : 1];  // FUSEQ: 1/(dec(sf) xg) per scale byte
+        float c6 = 0.0f;
         if constexpr (C::FUSEQ) {
             if (p.xnpart != 0) {  // the computed tensor scale: amax / 2688
                 float m = 0.0f;
@@ -836,6 +839,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 xg = *p.g_w;  // swapped form: g_w is the activations' slot, g_a the weights'
             }
             gg = __fmul_rn(xg, *p.g_a);
+            c6 = nvfp4_fast_c6(xg);
+            for (int i = et; i < 256; i += C::EPI_WARPS * 32)
+                s_rcp[i] = nvfp4_block_rcp((uint32_t)i, xg);
             // scale-atom rows past the 16 activation rows: zero once in every stage
             for (int s = 0; s < C::STAGES; ++s) {
                 uint8_t *sfb = smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES + C::SFA_BYTES;
@@ -873,7 +879,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (!(okq = warp_wait(&empty[qstage], qphase ^ 1u, abort, lane)))
                         break;
                     uint8_t *sB = smem + qstage * C::STAGE_BYTES + C::A_BYTES;
-                    fuseq_store(p, sB, sB + C::B_BYTES + C::SFA_BYTES, kt, et, cur, xg);
+                    fuseq_store(p, sB, sB + C::B_BYTES + C::SFA_BYTES, kt, et, cur, xg, c6, s_rcp);
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
                     __syncwarp();
                     if (lane == 0)
