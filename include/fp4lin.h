@@ -117,8 +117,10 @@ int nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
  * (Blackwell's 5th-generation tensor cores apply the two-level scaling in
  * hardware); "FP8, NVFP4 czy AWQ?", section "Dlaczego W8A8 i W4A16 to nie to
  * samo?" (W4A4: weights and activations both 4-bit, the product on low-precision
- * tensor cores).  Result:
- * tensor cores, y = bf16_round(g_a * g_w * acc).
+ * tensor cores).  Result: y = bf16_round(g_a * g_w * acc).
+ * The library picks the kernel (CTA pairs over 256 x 256 tiles for M >= 256
+ * without a K split, else one CTA per tile; FP4LIN_GEMM_KERNEL=single or =pair
+ * forces one); every choice gives the same bytes.
  *   a_codes [M, K/2], a_scales tensor-core layout of [M, K/16];
  *   w_codes [N, K/2], w_scales tensor-core layout of [N, K/16];
  *   g_a, g_w device floats; y bf16 with row stride ldy elements.
