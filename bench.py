@@ -748,7 +748,10 @@ def main():
         r["traffic"] = NCU_TRAFFIC.get(k)
         if k in NCU_TRAFFIC_NOTE:
             r["traffic_note"] = NCU_TRAFFIC_NOTE[k]
-    rooflines["quantize"]["note"] = "2.5625 B/element (one read of A); the dynamic tensor scale reads A twice"
+    rooflines["quantize"]["note"] = ("2.5625 B/element (one read of A); the dynamic tensor scale reads A twice: "
+                                     "frac_of_bytes_moved counts the 4.5625 B/element the two passes move")
+    q_moved = w.quant_bytes() + 2.0 * w.M * w.K  # plus the second read of A
+    rooflines["quantize"]["frac_of_bytes_moved"] = q_moved / (q_ms * 1e-3) / 1e9 / hbm
     rooflines["kv_load_fp8"]["frac_of_8tbs"] = rooflines["kv_load_fp8"]["achieved"] / 8000.0
     shares = {"quantize": q_ms, "gemm": gemm_ms, "kv_store": st_ms, "kv_load_fp8": ld_ms}
     dominant = max(shares, key=shares.get)
@@ -758,6 +761,7 @@ def main():
     roof["kernels"] = {k: {"achieved": r["achieved"], "peak": r["peak"], "unit": r["unit"], "frac": r["frac"],
                            "ms": r["ms"]} for k, r in rooflines.items()}
     roof["kernels"]["gemm"]["frac_of_clock_fp4"] = gemm_tf / clock_fp4
+    roof["kernels"]["quantize"]["frac_of_bytes_moved"] = rooflines["quantize"]["frac_of_bytes_moved"]
     roof["kernels"]["mxfp4_gemm"]["frac_of_clock_fp4"] = mx_gemm_tf / clock_fp4
     roof["kernels"]["mxfp4_gemm"]["layer_tflops"] = flops / (mx_ms * 1e-3) / 1e12
     roof["kernels"]["mxfp4_gemm"]["rel_frobenius_error"] = c3_err
